@@ -1,0 +1,330 @@
+"""Seeded synthetic inputs for the DSA decode path.
+
+This module is shared by the CUDA path's tests/benchmark and by the fp64 oracle's
+tests. It holds no arithmetic of the method itself: it only draws random numbers,
+quantises them to the storage formats (bf16 bits, OCP FP8 E4M3 codes with fp32
+scales), plants "hot" tokens and lays the caches out through a paged block table.
+
+Workload shapes follow the five workloads of the DeepSeek-Sparse-Attention decode
+hot path (lightning indexer -> top-k + page map -> MLA sparse decode) named on
+"GLM-52 Runs on RTX 4090" (kernel list) and the glm-5.2-4090 README ("how it works"):
+
+  cfg0  tiny bf16 decode      B=1,  L=4096,       top_k=256
+  cfg1  batched fp8 decode    B=8,  L=32768 each, top_k=2048
+  cfg2  serving-shaped decode B=64, L_b ~ U{2048..65536}, shared page pool
+  cfg3  long-context decode   B=1,  L=1,048,576, 256 log-uniform hot tokens
+  cfg4  chunked prefill       1 sequence, L=65536, 2048 causal queries
+
+Random streams: every tensor chunk has its own numpy PCG64 stream keyed by
+(seed, tensor id, row, chunk), so the bytes do not depend on the thread count.
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import numpy as np
+import torch
+
+PAGE = 64          # tokens per page
+H = 64             # heads (indexer and MLA)
+DI = 128           # indexer head dim
+DK = 576           # MLA key width: 512 latent + 64 rope
+DV = 512           # MLA value width
+KV_GROUPS = 5      # fp8 MLA scale groups: 4 x 128 latent columns + the 64 rope columns
+FP8_MAX = 448.0
+
+_POISON_SCALE = 1.0e4
+_FP8_POISON = 0x7E          # +448, the largest finite E4M3 code
+_CHUNK_TOKENS = 32768       # tokens per generation chunk
+
+
+@dataclass(frozen=True)
+class CaseSpec:
+    """One synthetic workload. All sizes are in tokens unless stated."""
+    name: str
+    seq_lens: tuple                  # per-sequence cache lengths
+    top_k: int
+    idx_dtype: str = "fp8"           # "bf16" | "fp8": indexer q and key cache
+    kv_dtype: str = "fp8"            # "bf16" | "fp8": MLA latent cache
+    out_dtype: str = "bf16"          # "fp32" | "bf16"
+    n_q: int = 1                     # queries per sequence (1 = decode)
+    q_pos: Optional[tuple] = None    # causal positions of the n_q queries of a sequence
+    n_planted: int = 32              # hot tokens per sequence (decode only)
+    planted_mode: str = "uniform"    # "uniform" | "loguniform"
+    seed: int = 0
+    extra_pages: int = 0             # unused physical pages (filled with poison)
+    max_pages: Optional[int] = None  # block-table width (default: longest sequence)
+    softmax_scale: float = 1.0 / math.sqrt(192.0)
+    kv_std: float = 0.5
+
+    @property
+    def B(self) -> int:
+        return len(self.seq_lens)
+
+    @property
+    def Bq(self) -> int:
+        return self.B * self.n_q
+
+
+def _cfg2_lens(seed: int) -> tuple:
+    rng = np.random.default_rng(np.random.SeedSequence(seed, spawn_key=(99,)))
+    return tuple(int(x) for x in rng.integers(2048, 65536, size=64, endpoint=True))
+
+
+CONFIGS = {
+    "cfg0": CaseSpec("cfg0", (4096,), top_k=256, idx_dtype="bf16", kv_dtype="bf16",
+                     out_dtype="fp32", n_planted=32, seed=0),
+    "cfg1": CaseSpec("cfg1", (32768,) * 8, top_k=2048, n_planted=32, seed=1),
+    "cfg2": CaseSpec("cfg2", _cfg2_lens(2), top_k=2048, n_planted=32, seed=2),
+    "cfg3": CaseSpec("cfg3", (1048576,), top_k=2048, n_planted=256,
+                     planted_mode="loguniform", seed=3),
+    "cfg4": CaseSpec("cfg4", (65536,), top_k=2048, n_q=2048,
+                     q_pos=tuple(range(63488, 65536)), n_planted=0, seed=4),
+}
+
+WORKLOAD_NAMES = {
+    "cfg0": "tiny bf16 decode B=1 L=4096 top_k=256",
+    "cfg1": "batched fp8 decode B=8 L=32768 top_k=2048",
+    "cfg2": "serving-shaped fp8 decode B=64 L~U[2048,65536] top_k=2048",
+    "cfg3": "long-context fp8 decode B=1 L=1048576 top_k=2048",
+    "cfg4": "chunked-prefill fp8 n_q=2048 at 63488..65535 of L=65536 top_k=2048",
+}
+
+
+def spec(name: str, **overrides) -> CaseSpec:
+    s = CONFIGS[name]
+    return replace(s, **overrides) if overrides else s
+
+
+# ----------------------------------------------------------------------------------
+# storage-format helpers (library conversions only)
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns (round-to-nearest-even, via torch)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def to_e4m3_codes(x: np.ndarray) -> np.ndarray:
+    """float32 already in code units -> OCP E4M3 ("fn") codes, RNE, saturated to +-448."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).clamp_(-FP8_MAX, FP8_MAX)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def quantize_rows_e4m3(x: np.ndarray):
+    """Per-row amax/448 scaling along the last axis -> (codes, fp32 scales)."""
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / FP8_MAX, 1.0).astype(np.float32)
+    codes = to_e4m3_codes(x / scale[..., None])
+    return codes, scale
+
+
+def _rng(seed: int, *key) -> np.random.Generator:
+    return np.random.default_rng(np.random.SeedSequence(seed, spawn_key=tuple(key)))
+
+
+def _threads() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+# ----------------------------------------------------------------------------------
+
+def _planted_positions(s: CaseSpec, b: int, L: int) -> np.ndarray:
+    n = min(s.n_planted, L) if s.n_q == 1 else 0
+    if n <= 0:
+        return np.zeros(0, dtype=np.int64)
+    rng = _rng(s.seed, 7, b)
+    if s.planted_mode == "loguniform":
+        picked: list = []
+        seen = set()
+        while len(picked) < n:
+            p = int(math.floor(math.exp(rng.uniform(0.0, math.log(L)))))
+            p = min(max(p, 0), L - 1)
+            if p not in seen:
+                seen.add(p)
+                picked.append(p)
+        return np.array(sorted(picked), dtype=np.int64)
+    return np.sort(rng.choice(L, size=n, replace=False)).astype(np.int64)
+
+
+def generate(s: CaseSpec) -> dict:
+    """Build every input of one workload as host numpy arrays.
+
+    Returned keys (shapes; Bq = B * n_q; P = physical pages):
+      seq_lens int32 [B], q_pos int32 [Bq] or None, block_table int32 [B, max_pages]
+      (unused entries -1), num_pages, page_size,
+      q_idx uint16 bf16-bits or uint8 e4m3 codes [Bq, 64, 128], q_idx_scale f32 [Bq, 64] or None,
+      head_w f32 [Bq, 64],
+      k_cache uint16 / uint8 [P, 64, 128], k_scale f32 [P, 64] or None,
+      q_mla uint16 bf16-bits [Bq, 64, 576],
+      kv_cache uint16 / uint8 [P*64, 576], kv_scale f32 [P*64, 5] or None,
+      planted: list of int64 arrays (logical hot-token positions per sequence).
+    """
+    B, n_q, Bq = s.B, s.n_q, s.Bq
+    lens = np.asarray(s.seq_lens, dtype=np.int64)
+    pages_per = (lens + PAGE - 1) // PAGE
+    used_pages = int(pages_per.sum())
+    P = used_pages + s.extra_pages
+    max_pages = int(s.max_pages if s.max_pages is not None else max(1, int(pages_per.max(initial=1))))
+    if max_pages < int(pages_per.max(initial=0)):
+        raise ValueError("max_pages smaller than the longest sequence")
+
+    # shared pool of shuffled pages handed out to sequences in order
+    perm = _rng(s.seed, 1).permutation(P).astype(np.int32)
+    bt = np.full((B, max_pages), -1, dtype=np.int32)
+    off = 0
+    for b in range(B):
+        n = int(pages_per[b])
+        bt[b, :n] = perm[off:off + n]
+        off += n
+
+    q_pos = None
+    if s.q_pos is not None:
+        if len(s.q_pos) != n_q:
+            raise ValueError("q_pos must list n_q positions")
+        q_pos = np.tile(np.asarray(s.q_pos, dtype=np.int32), B)
+
+    # ---- indexer queries and head weights
+    rq = _rng(s.seed, 2)
+    qf = (rq.standard_normal((Bq, H, DI), dtype=np.float32) / np.float32(math.sqrt(DI)))
+    head_w = (rq.uniform(0.0, 1.0, size=(Bq, H)).astype(np.float32) / np.float32(64.0))
+    if s.idx_dtype == "bf16":
+        q_idx, q_idx_scale = to_bf16_bits(qf), None
+    else:
+        q_idx, q_idx_scale = quantize_rows_e4m3(qf)
+
+    # ---- MLA queries (already absorbed, post-RoPE): N(0,1) in bf16
+    q_mla = to_bf16_bits(_rng(s.seed, 3).standard_normal((Bq, H, DK), dtype=np.float32))
+
+    # ---- caches, poisoned by default (tails of last pages and unused pages)
+    if s.idx_dtype == "bf16":
+        k_cache = np.full((P, PAGE, DI), to_bf16_bits(np.float32([_POISON_SCALE]))[0], dtype=np.uint16)
+        k_scale = None
+    else:
+        k_cache = np.full((P, PAGE, DI), _FP8_POISON, dtype=np.uint8)
+        k_scale = np.full((P, PAGE), _POISON_SCALE, dtype=np.float32)
+    if s.kv_dtype == "bf16":
+        kv_cache = np.full((P * PAGE, DK), to_bf16_bits(np.float32([_POISON_SCALE]))[0], dtype=np.uint16)
+        kv_scale = None
+    else:
+        kv_cache = np.full((P * PAGE, DK), _FP8_POISON, dtype=np.uint8)
+        kv_scale = np.full((P * PAGE, KV_GROUPS), _POISON_SCALE, dtype=np.float32)
+
+    planted = [_planted_positions(s, b, int(lens[b])) for b in range(B)]
+    # planting direction u_b = normalize(sum_h w[h] q_idx[h]) of the sequence's (single) query
+    dirs = []
+    for b in range(B):
+        if n_q == 1 and planted[b].size:
+            v = (head_w[b][:, None] * qf[b]).sum(axis=0)
+            dirs.append(v / np.linalg.norm(v))
+        else:
+            dirs.append(None)
+    shift = np.float32(3.0 / math.sqrt(DI))
+
+    tasks = []
+    for b in range(B):
+        L = int(lens[b])
+        for c0 in range(0, L, _CHUNK_TOKENS):
+            tasks.append((b, c0, min(L, c0 + _CHUNK_TOKENS)))
+
+    def fill(task):
+        b, t0, t1 = task
+        n = t1 - t0
+        # physical slot of every logical token in [t0, t1)
+        tok = np.arange(t0, t1)
+        phys = bt[b, tok // PAGE].astype(np.int64) * PAGE + (tok % PAGE)
+        ci = t0 // _CHUNK_TOKENS
+        # indexer keys
+        kf = _rng(s.seed, 4, b, ci).standard_normal((n, DI), dtype=np.float32) / np.float32(math.sqrt(DI))
+        if dirs[b] is not None:
+            sel = planted[b][(planted[b] >= t0) & (planted[b] < t1)] - t0
+            kf[sel] += shift * dirs[b][None, :].astype(np.float32)
+        kflat = k_cache.reshape(P * PAGE, DI)
+        if s.idx_dtype == "bf16":
+            kflat[phys] = to_bf16_bits(kf)
+        else:
+            codes, sc = quantize_rows_e4m3(kf)
+            kflat[phys] = codes
+            k_scale.reshape(-1)[phys] = sc
+        # MLA latent cache
+        vf = _rng(s.seed, 5, b, ci).standard_normal((n, DK), dtype=np.float32) * np.float32(s.kv_std)
+        if s.kv_dtype == "bf16":
+            kv_cache[phys] = to_bf16_bits(vf)
+        else:
+            groups = [vf[:, g * 128:(g + 1) * 128] for g in range(4)] + [vf[:, 512:576]]
+            codes = np.empty((n, DK), dtype=np.uint8)
+            scs = np.empty((n, KV_GROUPS), dtype=np.float32)
+            for g, blk in enumerate(groups):
+                c, sc = quantize_rows_e4m3(blk)
+                lo = g * 128
+                codes[:, lo:lo + blk.shape[1]] = c
+                scs[:, g] = sc
+            kv_cache[phys] = codes
+            kv_scale[phys] = scs
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(fill, tasks))
+
+    return dict(
+        spec=s, B=B, n_q=n_q, Bq=Bq, page_size=PAGE, num_pages=P, max_pages=max_pages,
+        seq_lens=lens.astype(np.int32), q_pos=q_pos, block_table=bt,
+        q_idx=q_idx, q_idx_scale=q_idx_scale, head_w=head_w,
+        k_cache=k_cache, k_scale=k_scale,
+        q_mla=q_mla, kv_cache=kv_cache, kv_scale=kv_scale,
+        top_k=s.top_k, softmax_scale=float(np.float32(s.softmax_scale)),
+        idx_dtype=s.idx_dtype, kv_dtype=s.kv_dtype, out_dtype=s.out_dtype,
+        planted=planted,
+    )
+
+
+def vis_lengths(case: dict) -> np.ndarray:
+    """Visible prefix length of every query: q_pos+1 when causal, else the sequence length.
+
+    This is part of the inputs' definition (which tokens a query may see), not of the method."""
+    if case["q_pos"] is not None:
+        return case["q_pos"].astype(np.int64) + 1
+    return np.repeat(case["seq_lens"].astype(np.int64), case["n_q"])
+
+
+def algorithmic_bytes(case: dict) -> dict:
+    """Bytes the decode step must move: every visited indexer key once, every selected
+    MLA row once, every query-side input once and the output once."""
+    vis = vis_lengths(case)
+    ik = 2 * DI if case["idx_dtype"] == "bf16" else DI + 4
+    kvb = 2 * DK if case["kv_dtype"] == "bf16" else DK + 4 * KV_GROUPS
+    # unique indexer-key bytes: every token of every sequence is read once per call
+    lens = case["seq_lens"].astype(np.int64)
+    idx_bytes = int(lens.sum()) * ik + int(((lens + PAGE - 1) // PAGE).sum()) * 4
+    sel = np.minimum(vis, case["top_k"])
+    mla_bytes = int(sel.sum()) * kvb
+    qb = (2 if case["idx_dtype"] == "bf16" else 1) * H * DI + (0 if case["idx_dtype"] == "bf16" else 4 * H)
+    ob = (4 if case["out_dtype"] == "fp32" else 2) * H * DV
+    q_bytes = case["Bq"] * (qb + 4 * H + 2 * H * DK + ob)
+    return dict(indexer=idx_bytes, mla=mla_bytes, query_side=q_bytes,
+                total=idx_bytes + mla_bytes + q_bytes)
+
+
+def to_torch(case: dict, device="cuda") -> dict:
+    """Host numpy arrays -> torch tensors on `device` (bf16 bits become torch.bfloat16,
+    E4M3 codes become torch.float8_e4m3fn). Plumbing only."""
+    def t(a, kind=None):
+        if a is None:
+            return None
+        x = torch.from_numpy(np.ascontiguousarray(a))
+        if kind == "bf16":
+            x = x.view(torch.int16).view(torch.bfloat16)
+        elif kind == "fp8":
+            x = x.view(torch.float8_e4m3fn)
+        return x.to(device)
+    idk = "bf16" if case["idx_dtype"] == "bf16" else "fp8"
+    kvk = "bf16" if case["kv_dtype"] == "bf16" else "fp8"
+    return dict(
+        seq_lens=t(case["seq_lens"]), q_pos=t(case["q_pos"]), block_table=t(case["block_table"]),
+        q_idx=t(case["q_idx"], idk), q_idx_scale=t(case["q_idx_scale"]), head_w=t(case["head_w"]),
+        k_cache=t(case["k_cache"], idk), k_scale=t(case["k_scale"]),
+        q_mla=t(case["q_mla"], "bf16"), kv_cache=t(case["kv_cache"], kvk), kv_scale=t(case["kv_scale"]),
+    )

@@ -1,0 +1,269 @@
+"""fp64 CPU oracle for the DeepSeek-Sparse-Attention (DSA) decode step.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or execute
+this module: only tests/, __graft_entry__.smoke() and bench.py's CPU-baseline /
+reference arm use it. It shares no code with the CUDA library.
+
+What it computes, stage by stage, in the order the pages name the kernels
+("GLM-52 Runs on RTX 4090", kernel list: lightning-indexer GEMM, top-k +
+page-mapping transforms, MLA sparse decode; glm-5.2-4090 README, "how it works"):
+
+  1. indexer_scores     score[q,s] = sum_h w[q,h] * ReLU(q_idx[q,h] . k_idx[s])  for s < vis(q)
+  2. topk_logical       the min(top_k, vis(q)) highest-scoring logical token indices
+  3. pagemap            logical token -> physical cache slot through the block table
+  4. mla_sparse_attention  64-head softmax attention over only the selected rows of the
+                        576-wide latent cache (keys: all 576 columns, values: first 512)
+                        ("Show HN: colibri", features: compressed KV of 576 floats per
+                        token, 64 heads, no GQA)
+
+Every stored code is decoded exactly to fp64 (own E4M3 and bf16 decoders, from the
+OCP 8-bit floating point definition and the bfloat16 bit layout) and multiplied by
+its fp32 scale; all arithmetic after that is fp64.
+
+Readings of points the pages leave open (each one is listed in the design notes):
+  * the indexer has no extra 1/sqrt(d) factor, ReLU comes before the head weights;
+  * fp8 indexer queries carry one fp32 scale per (query, head); fp8 indexer keys one
+    fp32 scale per token; fp8 latent rows five fp32 scales, one per 128-column group of
+    the 512 latent columns plus one for the 64 rope columns;
+  * ties in top-k go to the lower logical index; output is in descending-score order;
+  * with vis(q) <= top_k every visible token is selected (the dense path);
+  * an empty selection gives a zero output and lse = -inf.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+PAGE = 64
+H = 64
+DI = 128
+DK = 576
+DV = 512
+
+
+# ----------------------------------------------------------------------------------
+# storage formats
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """OCP FP8 E4M3 ("fn" variant) code -> exact fp64 value.
+
+    1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits. Exponent field 0 is
+    subnormal (value = m/8 * 2^-6). There is no infinity; S.1111.111 is NaN, so the
+    largest finite magnitude is 1.75 * 2^8 = 448."""
+    c = np.asarray(codes).astype(np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = np.ldexp(1.0 + m / 8.0, (e - 7).astype(np.int64))
+    sub = np.ldexp(m / 8.0, -6)
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 0xF) & ((c & 0x7) == 0x7), np.nan, v)
+
+
+def decode_bf16(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit pattern -> exact fp64 value (bf16 is the top half of an IEEE fp32)."""
+    b = np.asarray(bits).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _decode(codes: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return decode_bf16(codes)
+    if dtype == "fp8":
+        return decode_e4m3(codes)
+    raise ValueError(dtype)
+
+
+def dequant_index_queries(case: dict) -> np.ndarray:
+    """q_idx [Bq, 64, 128] as fp64: code value times its per-(query, head) scale."""
+    q = _decode(case["q_idx"], case["idx_dtype"])
+    if case["q_idx_scale"] is not None:
+        q = q * case["q_idx_scale"].astype(np.float64)[:, :, None]
+    return q
+
+
+def dequant_index_keys(case: dict, slots: np.ndarray) -> np.ndarray:
+    """Indexer keys of the given physical slots, [n, 128] fp64 (per-token scale applied)."""
+    flat = case["k_cache"].reshape(-1, DI)
+    k = _decode(flat[slots], case["idx_dtype"])
+    if case["k_scale"] is not None:
+        k = k * case["k_scale"].reshape(-1).astype(np.float64)[slots][:, None]
+    return k
+
+
+def dequant_latent_rows(case: dict, slots: np.ndarray) -> np.ndarray:
+    """Latent KV rows of the given physical slots, [n, 576] fp64.
+
+    fp8 rows: column group g in {0..3} covers columns [128g, 128g+128) and group 4 the
+    64 rope columns [512, 576); each group has its own fp32 scale per row."""
+    kv = _decode(case["kv_cache"][slots], case["kv_dtype"])
+    if case["kv_scale"] is not None:
+        sc = case["kv_scale"][slots].astype(np.float64)
+        col_group = np.minimum(np.arange(DK) // 128, 4)
+        kv = kv * sc[:, col_group]
+    return kv
+
+
+# ----------------------------------------------------------------------------------
+# paging
+
+def visible_lengths(case: dict) -> np.ndarray:
+    """vis(q): q_pos[q] + 1 for causal queries, else the sequence length of q's row."""
+    if case.get("q_pos") is not None:
+        return case["q_pos"].astype(np.int64) + 1
+    return np.repeat(case["seq_lens"].astype(np.int64), case["n_q"])
+
+
+def physical_slots(block_table_row: np.ndarray, logical: np.ndarray) -> np.ndarray:
+    """Page-mapping transform of one row: slot = table[i // 64] * 64 + i % 64; -1 stays -1."""
+    logical = np.asarray(logical, dtype=np.int64)
+    out = np.full(logical.shape, -1, dtype=np.int64)
+    ok = logical >= 0
+    li = logical[ok]
+    out[ok] = block_table_row[li // PAGE].astype(np.int64) * PAGE + li % PAGE
+    return out
+
+
+def pagemap(case: dict, logical: np.ndarray) -> np.ndarray:
+    """[Bq, top_k] logical token indices -> physical slots (query q uses row q // n_q)."""
+    out = np.empty(logical.shape, dtype=np.int64)
+    for q in range(logical.shape[0]):
+        out[q] = physical_slots(case["block_table"][q // case["n_q"]], logical[q])
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# stage 1: lightning indexer
+
+def indexer_scores(case: dict, queries=None) -> np.ndarray:
+    """score[q, s] = sum_h w[q,h] * max(0, <q_idx[q,h], k_idx[s]>) for s < vis(q), else -inf.
+
+    Returns fp64 [len(queries), L_max] with L_max = max_pages * 64. `queries` selects a
+    subset of the Bq query rows (default: all)."""
+    Bq = case["Bq"]
+    queries = np.arange(Bq) if queries is None else np.asarray(queries)
+    L_max = case["max_pages"] * PAGE
+    vis = visible_lengths(case)
+    Q = dequant_index_queries(case)
+    w = case["head_w"].astype(np.float64)
+    out = np.full((len(queries), L_max), -np.inf)
+    for i, q in enumerate(queries):
+        v = int(vis[q])
+        if v == 0:
+            continue
+        slots = physical_slots(case["block_table"][q // case["n_q"]], np.arange(v))
+        K = dequant_index_keys(case, slots)                 # [v, 128]
+        logits = Q[q] @ K.T                                  # [64, v]
+        out[i, :v] = (w[q][:, None] * np.maximum(logits, 0.0)).sum(axis=0)
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# stage 2: top-k selection
+
+def topk_logical(scores: np.ndarray, vis: np.ndarray, top_k: int) -> np.ndarray:
+    """Per query, the min(top_k, vis) largest scores among tokens [0, vis).
+
+    Order: descending score, ties to the lower index (a stable sort). Unused entries -1.
+    With vis <= top_k this is every visible token (the dense path)."""
+    n = scores.shape[0]
+    out = np.full((n, top_k), -1, dtype=np.int64)
+    for i in range(n):
+        v = int(vis[i])
+        k = min(top_k, v)
+        if k == 0:
+            continue
+        idx = np.arange(v)
+        order = np.lexsort((idx, -scores[i, :v]))   # primary: -score, secondary: index
+        out[i, :k] = idx[order[:k]]
+    return out
+
+
+# ----------------------------------------------------------------------------------
+# stage 3: MLA sparse attention (+ the split-KV combine)
+
+def mla_sparse_attention(case: dict, physical: np.ndarray, queries=None):
+    """out[q,h,:] = sum_j softmax_j(z[q,h,:]) * V[slot_j], z = scale * <q_mla[q,h], K[slot_j]>.
+
+    K = all 576 columns of the selected latent rows, V = their first 512 columns.
+    physical: [n, top_k] slots (-1 = unused). Returns (out fp64 [n, 64, 512],
+    lse fp64 [n, 64]) with lse = log sum_j exp(z_j); an empty selection gives 0 and -inf."""
+    queries = np.arange(physical.shape[0]) if queries is None else np.asarray(queries)
+    scale = float(case["softmax_scale"])
+    out = np.zeros((len(queries), H, DV))
+    lse = np.full((len(queries), H), -np.inf)
+    for i, q in enumerate(queries):
+        sel = physical[i][physical[i] >= 0]
+        if sel.size == 0:
+            continue
+        qm = decode_bf16(case["q_mla"][q])                   # [64, 576]
+        KV = dequant_latent_rows(case, sel)                  # [n, 576]
+        z = scale * (qm @ KV.T)                              # [64, n]
+        m = z.max(axis=1, keepdims=True)
+        e = np.exp(z - m)
+        l = e.sum(axis=1, keepdims=True)
+        out[i] = (e / l) @ KV[:, :DV]
+        lse[i] = (m + np.log(l))[:, 0]
+    return out, lse
+
+
+def mla_partials(case: dict, slots: np.ndarray, q: int):
+    """Un-normalised attention state of one query over one subset of slots:
+    m[h] = max_j z, l[h] = sum_j exp(z - m), o[h] = sum_j exp(z - m) V_j."""
+    scale = float(case["softmax_scale"])
+    slots = slots[slots >= 0]
+    if slots.size == 0:
+        return np.full(H, -np.inf), np.zeros(H), np.zeros((H, DV))
+    qm = decode_bf16(case["q_mla"][q])
+    KV = dequant_latent_rows(case, slots)
+    z = scale * (qm @ KV.T)
+    m = z.max(axis=1)
+    e = np.exp(z - m[:, None])
+    return m, e.sum(axis=1), e @ KV[:, :DV]
+
+
+def combine_partials(ms, ls, os_):
+    """Log-sum-exp merge of split states: M = max_s m_s, a_s = exp(m_s - M),
+    out = sum_s a_s o_s / sum_s a_s l_s, lse = M + log(sum_s a_s l_s)."""
+    ms = np.stack(ms)            # [S, H]
+    ls = np.stack(ls)
+    os_ = np.stack(os_)          # [S, H, DV]
+    M = ms.max(axis=0)
+    Msafe = np.where(np.isfinite(M), M, 0.0)
+    a = np.where(np.isfinite(ms), np.exp(ms - Msafe[None, :]), 0.0)
+    L = (a * ls).sum(axis=0)
+    O = (a[:, :, None] * os_).sum(axis=0)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(L[:, None] > 0, O / np.where(L > 0, L, 1.0)[:, None], 0.0)
+        lse = np.where(L > 0, Msafe + np.log(np.where(L > 0, L, 1.0)), -np.inf)
+    return out, lse
+
+
+def mla_sparse_attention_split(case: dict, physical: np.ndarray, n_splits: int, queries=None):
+    """Same result as mla_sparse_attention, computed as n_splits contiguous chunks of the
+    index list merged by combine_partials (the split-KV reduction)."""
+    queries = np.arange(physical.shape[0]) if queries is None else np.asarray(queries)
+    out = np.zeros((len(queries), H, DV))
+    lse = np.full((len(queries), H), -np.inf)
+    for i, q in enumerate(queries):
+        parts = np.array_split(physical[i], n_splits)
+        st = [mla_partials(case, p, q) for p in parts]
+        out[i], lse[i] = combine_partials([s[0] for s in st], [s[1] for s in st], [s[2] for s in st])
+    return out, lse
+
+
+# ----------------------------------------------------------------------------------
+# the whole step
+
+def decode_layer(case: dict, queries=None):
+    """Indexer -> top-k -> page map -> MLA sparse attention for the chosen query rows.
+
+    Returns dict(scores, logical, physical, out, lse), all fp64 / int64."""
+    queries = np.arange(case["Bq"]) if queries is None else np.asarray(queries)
+    scores = indexer_scores(case, queries)
+    vis = visible_lengths(case)[queries]
+    logical = topk_logical(scores, vis, case["top_k"])
+    phys = np.empty_like(logical)
+    for i, q in enumerate(queries):
+        phys[i] = physical_slots(case["block_table"][q // case["n_q"]], logical[i])
+    out, lse = mla_sparse_attention(case, phys, queries)
+    return dict(scores=scores, logical=logical, physical=phys, out=out, lse=lse)
