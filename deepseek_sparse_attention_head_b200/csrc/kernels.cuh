@@ -1,0 +1,69 @@
+// Argument blocks and host launchers of the sm_100a kernels (one translation unit per stage).
+#pragma once
+
+#include "common.cuh"
+
+namespace dsa {
+
+struct IndexerArgs {
+  int B, n_q;
+  const int32_t* seq_lens;
+  const int32_t* q_pos;
+  const int32_t* block_table;
+  int max_pages;
+  int num_pages;
+  const float* q_scale;
+  const float* head_w;
+  const float* k_scale;
+  float* scores;
+  int64_t L_max;
+  const int32_t* tile_prefix;  // [B+1] exclusive prefix of ceil(len/128)
+  unsigned int* err;
+};
+
+struct TopkArgs {
+  int n_q;
+  const int32_t* seq_lens;
+  const int32_t* q_pos;
+  const int32_t* block_table;
+  int max_pages;
+  int num_pages;
+  const float* scores;
+  int64_t L_max;
+  int top_k;
+  int32_t* logical;   // may be null
+  int32_t* physical;  // may be null
+  unsigned int* err;
+};
+
+struct MlaArgs {
+  int Bq;
+  int top_k;
+  int nsplit;
+  int keys_per_split;   // multiple of 64
+  const uint8_t* kv;    // [num_slots, 576] fp8 codes or bf16 values
+  const float* kv_scale;
+  int64_t num_slots;
+  const int32_t* physical;
+  float scale_log2;     // softmax_scale * log2(e)
+  void* out;
+  int out_fp32;
+  float* lse;
+  float* part_ml;       // [Bq, nsplit, 64, 2]
+  float* part_o;        // [Bq, nsplit, 64, 512]
+  unsigned int* err;
+};
+
+// Each returns the launch error (cudaSuccess when queued) and adds the number of
+// kernels it queued to *launches.
+cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages,
+                        int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches);
+cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,
+                           int grid, cudaStream_t stream, int* launches);
+cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches);
+cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
+                           int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,
+                           cudaStream_t stream, int* launches);
+cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
+
+}  // namespace dsa

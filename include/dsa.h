@@ -1,0 +1,200 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DeepSeek-Sparse-Attention decode library.
+ *
+ * The decode step has three stages, named on "GLM-52 Runs on RTX 4090" (kernel list:
+ * 1. lightning-indexer GEMM, 2. top-k + page-mapping transforms, 3. MLA sparse decode)
+ * and in the renning22/glm-5.2-4090 README ("how it works": indexer, top-k + page
+ * mapping, MLA sparse decode; "usage": SGLANG_NSA_FUSE_TOPK=1 fuses the page-mapping
+ * transform into top-k):
+ *
+ *   score[q,s] = sum_h w[q,h] * ReLU(q_idx[q,h] . k_idx[s])            (64 heads x 128)
+ *   sel[q]     = the min(top_k, vis(q)) highest-scoring logical tokens s < vis(q)
+ *   slot       = block_table[b, s / 64] * 64 + s % 64                  (page size 64)
+ *   out[q,h,:] = sum_j softmax_j(scale * q_mla[q,h] . KV[slot_j, 0:576]) * KV[slot_j, 0:512]
+ *
+ * The latent cache row is 576 wide: 512 latent ("nope") columns plus 64 RoPE columns;
+ * keys use all 576, values the first 512 ("Show HN: colibri", features: compressed
+ * KV-cache of 576 floats per token, 64 heads, no GQA).
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named as device pointers are caller-owned device memory on the current
+ *    device; the library never allocates or frees device memory.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t, 0 = legacy default).
+ *  - Argument errors return synchronously, before any launch, with no side effect.
+ *  - Problems only the device can see (a block-table entry outside [0, num_pages),
+ *    a sequence longer than its block-table row, a slot index outside the cache)
+ *    are clamped so no access leaves its buffer, and are recorded in a sticky error
+ *    word inside the workspace; read it with dsa_get_error(). Kernels never trap.
+ *    Every wait inside a kernel is bounded (about one second); a wait that runs out
+ *    records DSA_ERR_TIMEOUT and the kernel returns.
+ *  - The workspace must be zero-filled once before its first use (cudaMemset); the
+ *    library leaves it reusable. Calls sharing one workspace must be stream-ordered.
+ *  - Layouts are row-major and contiguous as annotated. "fp8" is OCP FP8 E4M3, the
+ *    "fn" variant (no infinities, largest finite value 448).
+ *  - Index lists hold -1 in unused entries. Within a query the order of selected
+ *    indices is unspecified.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* bad pointer, size, dtype or alignment (synchronous)        */
+  DSA_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (synchronous)  */
+  DSA_ERR_CUDA = 3,          /* a CUDA runtime call failed (synchronous)                   */
+  DSA_ERR_WORKSPACE = 4,     /* workspace NULL, too small or misaligned (synchronous)      */
+  DSA_ERR_DEVICE_BOUNDS = 5, /* device-side: an index or length was out of range, clamped  */
+  DSA_ERR_TIMEOUT = 6        /* device-side: a bounded wait ran out                        */
+} dsa_status;
+
+typedef enum {
+  DSA_BF16 = 0,
+  DSA_FP8_E4M3 = 1,
+  DSA_FP32 = 2
+} dsa_dtype;
+
+/* Which call a workspace is sized for (dsa_workspace_size). */
+typedef enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_PAGEMAP = 2,
+  DSA_OP_LAYER = 3
+} dsa_op;
+
+/*
+ * Paged cache description shared by the indexer, top-k, page-map and layer calls
+ * (the "page-mapping transforms" of "GLM-52 Runs on RTX 4090", kernel list item 2).
+ * One block table and one physical slot numbering serve both the indexer-key cache
+ * and the latent cache. Query q (0 <= q < B*n_q) belongs to sequence b = q / n_q.
+ */
+typedef struct {
+  int32_t B;                  /* sequences (block-table rows), >= 1                        */
+  int32_t n_q;                /* queries per sequence: 1 for decode, >1 for chunked prefill */
+  const int32_t* seq_lens;    /* device [B]: tokens in each sequence's cache               */
+  const int32_t* q_pos;       /* device [B*n_q] causal position (vis = q_pos+1) or NULL
+                                 (vis = seq_len)                                            */
+  const int32_t* block_table; /* device [B, max_pages_per_seq]: physical page of each
+                                 logical page; entries past a sequence's length unused      */
+  int32_t max_pages_per_seq;  /* block-table row width, >= 1                               */
+  int32_t page_size;          /* tokens per page; must be 64                               */
+  int32_t num_pages;          /* physical pages in the caches (bounds for the table)       */
+} dsa_paging;
+
+/*
+ * Stage 1 - lightning indexer ("GLM-52 Runs on RTX 4090", kernel list item 1).
+ *   score[q, s] = k_scale[slot(s)] * sum_h (head_w[q,h] * q_scale[q,h]) * ReLU(<q8[q,h], k8[slot(s)]>)
+ * which equals sum_h w * ReLU(q_idx . k_idx) on the dequantised values (scales > 0).
+ *  q_idx    device [B*n_q, 64, 128] in q_dtype (DSA_BF16 or DSA_FP8_E4M3)
+ *  q_scale  device [B*n_q, 64] fp32 per (query, head) scale; required for fp8, NULL for bf16
+ *  head_w   device [B*n_q, 64] fp32 head weights
+ *  k_cache  device [num_pages, 64, 128] in k_dtype (must equal q_dtype)
+ *  k_scale  device [num_pages, 64] fp32 per-token scale; required for fp8, NULL for bf16
+ *  scores   device [B*n_q, L_max] fp32 output; entries s < vis(q) are written, the rest
+ *           are left untouched. L_max >= max_pages_per_seq*64 is not required, but
+ *           vis(q) is clamped to L_max.
+ *  Alignment: q_idx, k_cache 16-byte aligned; L_max >= 1.
+ */
+dsa_status dsa_indexer_scores(const dsa_paging* paging,
+                              const void* q_idx, dsa_dtype q_dtype, const float* q_scale,
+                              const float* head_w,
+                              const void* k_cache, dsa_dtype k_dtype, const float* k_scale,
+                              float* scores, int64_t L_max,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Stage 2 - top-k selection with the fused page-mapping transform ("GLM-52 Runs on
+ * RTX 4090", kernel list item 2; glm-5.2-4090 README, usage: SGLANG_NSA_FUSE_TOPK=1).
+ * For each query picks the k = min(top_k, vis(q)) largest scores among s < vis(q)
+ * (all of them when vis(q) <= top_k: the dense path) and writes
+ *  logical_out  device [B*n_q, top_k] int32 logical token indices, or NULL
+ *  physical_out device [B*n_q, top_k] int32 physical slots block_table[b,s/64]*64+s%64
+ * Entries k..top_k-1 are -1. Equal scores at the boundary are broken arbitrarily.
+ *  scores  device [B*n_q, L_max] fp32 (as written by dsa_indexer_scores)
+ *  1 <= top_k <= 16384.
+ */
+dsa_status dsa_topk_pagemap(const dsa_paging* paging, const float* scores, int64_t L_max,
+                            int32_t top_k, int32_t* logical_out, int32_t* physical_out,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The page-mapping transform alone (the second half of stage 2), exposed so a caller
+ * can map an index list it chose itself:
+ *  physical[q, i] = block_table[b, logical[q,i] / 64] * 64 + logical[q,i] % 64, -1 -> -1.
+ *  logical, physical  device [B*n_q, top_k] int32. Bit-exact integer transform.
+ */
+dsa_status dsa_pagemap(const dsa_paging* paging, const int32_t* logical, int32_t top_k,
+                       int32_t* physical, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Stage 3 - MLA sparse decode ("GLM-52 Runs on RTX 4090", kernel list item 3):
+ * 64-head attention of each query over only its selected latent rows, split across
+ * SMs along the index list and merged with an online-softmax (log-sum-exp) combine.
+ *  q         device [Bq, 64, 576] bf16 (absorbed, post-RoPE query)
+ *  kv_cache  device [num_slots, 576] in kv_dtype: DSA_BF16, or DSA_FP8_E4M3 with
+ *  kv_scale  device [num_slots, 5] fp32: scale g covers columns [128g, 128g+128) for
+ *            g < 4 and the 64 rope columns [512, 576) for g = 4; NULL for bf16
+ *  physical  device [Bq, top_k] int32 slots, -1 = unused
+ *  out       device [Bq, 64, 512] in out_dtype (DSA_BF16 or DSA_FP32)
+ *  lse       device [Bq, 64] fp32 natural-log sum of exp(logits), or NULL
+ * A query with no valid slot gets out = 0 and lse = -inf.
+ * Workspace: mla_workspace_size(Bq, top_k).
+ */
+dsa_status mla_sparse_decode(int32_t Bq, const void* q, const void* kv_cache, dsa_dtype kv_dtype,
+                             const float* kv_scale, int64_t num_slots,
+                             const int32_t* physical, int32_t top_k, float softmax_scale,
+                             void* out, dsa_dtype out_dtype, float* lse,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The fused decode layer: indexer -> top-k + page map -> MLA sparse decode on one
+ * stream, intermediate scores and index lists kept in the workspace. Arguments as
+ * in the three stages above (q_idx and k_cache share idx_dtype). The scores row
+ * stride is max_pages_per_seq * 64.
+ *  logical_out, physical_out  optional device [B*n_q, top_k] int32 copies of the
+ *                             selection (NULL to skip)
+ * Workspace: dsa_workspace_size(paging, 0, top_k, DSA_OP_LAYER).
+ */
+dsa_status dsa_decode_layer(const dsa_paging* paging,
+                            const void* q_idx, dsa_dtype idx_dtype, const float* q_scale,
+                            const float* head_w, const void* k_cache, const float* k_scale,
+                            const void* q_mla, const void* kv_cache, dsa_dtype kv_dtype,
+                            const float* kv_scale,
+                            int32_t top_k, float softmax_scale,
+                            void* out, dsa_dtype out_dtype, float* lse,
+                            int32_t* logical_out, int32_t* physical_out,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace `op` needs for this paging (L_max only matters for DSA_OP_INDEXER
+ * and DSA_OP_TOPK, where it may be 0). Returns 0 when the arguments are invalid. */
+size_t dsa_workspace_size(const dsa_paging* paging, int64_t L_max, int32_t top_k, int32_t op);
+
+/* Bytes of workspace mla_sparse_decode needs for Bq queries and top_k slots each
+ * (depends on the current device's SM count). 0 when the arguments are invalid. */
+size_t mla_workspace_size(int32_t Bq, int32_t top_k);
+
+/* Number of KV splits mla_sparse_decode will use on the current device. */
+int32_t mla_num_splits(int32_t Bq, int32_t top_k);
+
+/* Synchronises `stream`, returns the sticky device error recorded in `workspace`
+ * (DSA_OK if none) and clears it. */
+dsa_status dsa_get_error(void* workspace, void* stream);
+
+/* Static description of a status code. Never NULL. */
+const char* dsa_status_string(dsa_status status);
+
+/* Number of kernel launches the most recent successful call on this host thread
+ * issued (for launch accounting). */
+int32_t dsa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H */

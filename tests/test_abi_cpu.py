@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+symbol include/dsa.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import deepseek_sparse_attention_head_b200 as dsa
+from deepseek_sparse_attention_head_b200 import _lib, _Paging
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(0x100000)      # never dereferenced: every call below fails validation first
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)) - {"if"})
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert "dsa_decode_layer" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(_lib, n), n
+    assert sorted(names) == dsa.exported_symbols()
+
+
+def paging(B=2, n_q=1, page_size=64, max_pages=4, num_pages=8, seq=FAKE, table=FAKE):
+    return _Paging(B, n_q, seq, None, table, max_pages, page_size, num_pages)
+
+
+def ws_ok(pg, op=dsa.DSA_OP_INDEXER, L=256, top_k=16):
+    return _lib.dsa_workspace_size(ctypes.byref(pg), L, top_k, op)
+
+
+def call_indexer(pg, qd=dsa.DSA_FP8_E4M3, kd=dsa.DSA_FP8_E4M3, qs=FAKE, ks=FAKE, ws_bytes=None, ws=FAKE, L=256):
+    if ws_bytes is None:
+        ws_bytes = ws_ok(pg) if pg is not None else 1 << 20
+    return _lib.dsa_indexer_scores(ctypes.byref(pg) if pg is not None else None, FAKE, qd, qs, FAKE, FAKE, kd, ks,
+                                   FAKE, L, ws, ws_bytes, None)
+
+
+def test_indexer_argument_errors():
+    pg = paging()
+    assert call_indexer(None) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(paging(B=0)) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(paging(page_size=32)) == dsa.DSA_ERR_UNSUPPORTED
+    assert call_indexer(paging(seq=None)) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(pg, qd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG            # dtype mismatch
+    assert call_indexer(pg, qs=None) == dsa.DSA_ERR_INVALID_ARG                      # fp8 needs scales
+    assert call_indexer(pg, qd=dsa.DSA_BF16, kd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG  # bf16 takes none
+    assert call_indexer(pg, qd=dsa.DSA_FP32, kd=dsa.DSA_FP32) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(pg, L=0) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(pg, ws_bytes=16) == dsa.DSA_ERR_WORKSPACE
+    assert call_indexer(pg, ws=None) == dsa.DSA_ERR_WORKSPACE
+    assert call_indexer(pg, ws=ctypes.c_void_p(0x100010)) == dsa.DSA_ERR_WORKSPACE   # misaligned
+
+
+def test_topk_and_pagemap_argument_errors():
+    pg = paging()
+    ws = ws_ok(pg, dsa.DSA_OP_TOPK)
+    assert _lib.dsa_topk_pagemap(ctypes.byref(pg), FAKE, 256, 0, FAKE, FAKE, FAKE, ws, None) == dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_topk_pagemap(ctypes.byref(pg), FAKE, 256, 16, None, None, FAKE, ws, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_topk_pagemap(ctypes.byref(pg), None, 256, 16, FAKE, FAKE, FAKE, ws, None) == \
+        dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_pagemap(ctypes.byref(pg), None, 16, FAKE, FAKE, 4096, None) == dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_pagemap(ctypes.byref(pg), FAKE, 0, FAKE, FAKE, 4096, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_mla_argument_errors():
+    def call(Bq=2, kvd=dsa.DSA_FP8_E4M3, kvs=FAKE, top_k=64, scale=0.07, outd=dsa.DSA_BF16, q=FAKE):
+        return _lib.mla_sparse_decode(Bq, q, FAKE, kvd, kvs, 1024, FAKE, top_k, scale, FAKE, outd, None, FAKE,
+                                      1 << 30, None)
+    assert call(Bq=0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(q=None) == dsa.DSA_ERR_INVALID_ARG
+    assert call(top_k=0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(top_k=16385) == dsa.DSA_ERR_INVALID_ARG
+    assert call(scale=-1.0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == dsa.DSA_ERR_INVALID_ARG
+    assert call(kvs=None) == dsa.DSA_ERR_INVALID_ARG
+    assert call(kvd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG
+    assert call(outd=dsa.DSA_FP8_E4M3) == dsa.DSA_ERR_INVALID_ARG
+    assert call(q=ctypes.c_void_p(0x100008)) == dsa.DSA_ERR_INVALID_ARG   # TMA needs 16-byte alignment
+
+
+def test_workspace_sizes_are_consistent():
+    pg = paging(B=3, n_q=2, max_pages=10)
+    a = ws_ok(pg, dsa.DSA_OP_INDEXER, 640, 0)
+    assert a >= 256 + 4 * 4 and a % 256 == 0
+    layer = _lib.dsa_workspace_size(ctypes.byref(pg), 0, 64, dsa.DSA_OP_LAYER)
+    # scores [6, 640] fp32 + two [6, 64] int32 lists at least
+    assert layer >= 256 + 6 * 640 * 4 + 2 * 6 * 64 * 4
+    assert _lib.dsa_workspace_size(ctypes.byref(pg), 0, 0, dsa.DSA_OP_LAYER) == 0     # invalid top_k
+    assert _lib.dsa_workspace_size(None, 0, 64, dsa.DSA_OP_LAYER) == 0
+    assert _lib.mla_workspace_size(0, 64) == 0
+    assert _lib.mla_workspace_size(4, 64) >= 256
+
+
+def test_status_strings():
+    for s in range(7):
+        assert dsa.dsa_status_string(s)
+    assert dsa.dsa_status_string(99) == "unknown status"
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        dsa._ptr(torch.zeros(4))
