@@ -1,0 +1,406 @@
+"""Benchmark of the DSA decode layer (lightning indexer -> top-k + page map -> MLA
+sparse decode) on one B200, or N independent replicas under torchrun.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg2] [--impl ours|reference]
+
+Prints one JSON line (rank 0). A step is one dsa_decode_layer call over the whole
+batch of the workload; inputs are resident in HBM and larger than L2.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import dsa_inputs  # noqa: E402
+
+METRIC = "DSA decode layer-calls/s and achieved HBM TB/s (indexer+top-k+MLA)"
+UNIT = "layer-calls/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="cfg2", choices=sorted(dsa_inputs.CONFIGS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=200)
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+
+def file_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+INDEXER_SOURCES = ["deepseek_sparse_attention_head_b200/csrc/indexer.cu",
+                   "deepseek_sparse_attention_head_b200/csrc/common.cuh"]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def committed_traffic():
+    """Per-launch DRAM bytes of the indexer kernel from the committed ncu summary, or None
+    when the summary is absent or was taken on different kernel sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "indexer_traffic.json")) as f:
+            d = json.load(f)
+        if d.get("sources_sha") != file_hash(INDEXER_SOURCES):
+            return None
+        return d
+    except (OSError, ValueError):
+        return None
+
+
+def run_ours(args, world, rank, local):
+    import deepseek_sparse_attention_head_b200 as dsa
+
+    case = dsa_inputs.generate(dsa_inputs.spec(args.workload))
+    nbytes = dsa_inputs.algorithmic_bytes(case)
+    t = dsa_inputs.to_torch(case, "cuda")
+    paging = dsa.Paging(t["seq_lens"], t["block_table"], case["num_pages"], case["n_q"], t["q_pos"])
+    Bq, K = case["Bq"], case["top_k"]
+    out_dt = torch.float32 if case["out_dtype"] == "fp32" else torch.bfloat16
+    out = torch.empty(Bq, 64, 512, dtype=out_dt, device="cuda")
+    lse = torch.empty(Bq, 64, dtype=torch.float32, device="cuda")
+    ws = dsa.alloc_workspace(dsa.dsa_workspace_size(paging, 0, K, dsa.DSA_OP_LAYER))
+    stream = torch.cuda.Stream()
+
+    def step():
+        dsa.dsa_decode_layer(paging, t["q_idx"], t["q_idx_scale"], t["head_w"], t["k_cache"], t["k_scale"],
+                             t["q_mla"], t["kv_cache"], t["kv_scale"], K, case["softmax_scale"], out, ws, lse=lse,
+                             stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    launches_per_step = dsa.dsa_last_launch_count()
+    err = dsa.dsa_get_error(ws, stream)
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the warm-up call")
+
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        stream.synchronize()
+
+    def run(n):
+        for _ in range(n):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+
+    with torch.cuda.stream(stream):
+        run(max(3, args.warmup))
+    stream.synchronize()
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run(args.steps)
+        ev1.record(stream)
+    ev1.synchronize()
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    err = dsa.dsa_get_error(ws, stream)
+    if err != 0:
+        raise RuntimeError(f"device error {err} during the timed region")
+
+    # ---- dominant kernel (indexer stage) timed alone, same stream, same inputs
+    scores = torch.empty(Bq, paging.L_layer, dtype=torch.float32, device="cuda")
+    ws_i = dsa.alloc_workspace(dsa.dsa_workspace_size(paging, paging.L_layer, 0, dsa.DSA_OP_INDEXER))
+    reps = max(20, min(2000, args.steps // 5))
+
+    def idx_call():
+        dsa.dsa_indexer_scores(paging, t["q_idx"], t["q_idx_scale"], t["head_w"], t["k_cache"], t["k_scale"],
+                               scores, ws_i, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            idx_call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            idx_call()
+        e1.record(stream)
+    e1.synchronize()
+    idx_ms = e0.elapsed_time(e1) / reps
+
+    # ---- end to end through the public API with host buffers
+    pin = {k: t[k].cpu().pin_memory() for k in ("q_idx", "q_idx_scale", "head_w", "q_mla", "seq_lens",
+                                                   "block_table") if t[k] is not None}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+    n_e2e = max(10, args.e2e_steps)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            for k, v in pin.items():
+                t[k].copy_(v, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+            host_lse.copy_(lse, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    peak, peak_kind = measured_peaks()
+    calls_per_s = world * args.steps / (ms_max / 1e3)
+    idx_achieved = nbytes["indexer"] / (idx_ms / 1e3) / 1e9
+    tr = committed_traffic()
+    result = {
+        "metric": METRIC,
+        "value": calls_per_s,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3 (indexer, fp32 accum) + bf16 (MLA, fp32 accum)",
+        "data": "synthetic (seeded; dsa_inputs)",
+        "config": {
+            "workload": f"{args.workload}: {dsa_inputs.WORKLOAD_NAMES[args.workload]}",
+            "B": case["B"], "n_q": case["n_q"], "sum_L": int(case["seq_lens"].sum()), "top_k": K,
+            "algorithmic_bytes_per_step": nbytes["total"],
+            "l2": f"inputs larger than L2 ({nbytes['total'] / 1e6:.0f} MB read per step > 126 MB)",
+            "launch": "cuda_graph" if graph is not None else "eager",
+            "parallelism": f"replicas x{world}",
+        },
+        "achieved_hbm_tbs": nbytes["total"] / (ms_max / args.steps / 1e3) / 1e12,
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "indexer (dsa_indexer_scores: plan + tcgen05 indexer)",
+            "achieved": idx_achieved,
+            "peak": peak,
+            "peak_kind": f"{peak_kind} hbm_gbs (burst copy)",
+            "unit": "GB/s",
+            "frac": idx_achieved / peak,
+            "traffic": None if tr is None else tr["bytes_per_launch"],
+            "algorithmic_bytes": nbytes["indexer"],
+            "duration_us": idx_ms * 1e3,
+        },
+        "e2e": {"value": world * n_e2e / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(case, budget_s=20.0)
+    if graph is not None:
+        del graph
+    return result
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline / reference arm)
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle_rows(case, rows, deadline=None):
+    import oracle
+    t0 = time.perf_counter()
+    done = 0
+    for r in rows:
+        oracle.decode_layer(case, queries=[r])
+        done += 1
+        if deadline is not None and time.perf_counter() - t0 > deadline:
+            break
+    return time.perf_counter() - t0, done
+
+
+def cpu_baseline(case, budget_s=20.0):
+    """The oracle as it stands on this host's cores, on whole query rows of the workload
+    until about budget_s of CPU work; scaled to layer-calls/s by the row count."""
+    rows = list(range(case["Bq"]))
+    dt, done = time_oracle_rows(case, rows, deadline=budget_s)
+    per_row = dt / done
+    return {"value": 1.0 / (per_row * case["Bq"]), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{done} of {case['Bq']} query rows (full indexer+top-k+MLA per row), {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 oracle on the host cores, same workload and unit. Each step
+    processes one whole query row (rows cycle through the batch); at most ~150 s in total."""
+    case = dsa_inputs.generate(dsa_inputs.spec(args.workload))
+    Bq = case["Bq"]
+    per_row, _ = time_oracle_rows(case, [0])
+    budget = 150.0
+    steps = args.steps
+    warm = min(args.warmup, 3)
+    n_fit = max(1, int(budget / max(per_row, 1e-3)) - warm)
+    timed = min(steps, n_fit)
+    time_oracle_rows(case, [i % Bq for i in range(warm)])
+    dt, done = time_oracle_rows(case, [i % Bq for i in range(timed)])
+    value = done / Bq / dt
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": dt / done * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded; dsa_inputs)",
+        "config": {"workload": f"{args.workload}: {dsa_inputs.WORKLOAD_NAMES[args.workload]}",
+                   "B": case["B"], "n_q": case["n_q"], "top_k": case["top_k"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"{done} whole query rows timed (of {steps} requested steps; one row per step, "
+                                   f"rows cycle through the {Bq}-row batch)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return 0
+    world, rank, local = dist_setup(args)
+    res = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -77,11 +77,12 @@ dsa_status check_paging(const dsa_paging* pg) {
 
 int mla_splits_for(int Bq, int top_k, int* keys_per_split) {
   const int sms = device_sms();
-  const int ntiles = (top_k + 63) / 64;
+  const int tile = mla_tile_keys();
+  const int ntiles = (top_k + tile - 1) / tile;
   int s = sms > 0 ? sms / (Bq > 0 ? Bq : 1) : 1;
   if (s < 1) s = 1;
   if (s > ntiles) s = ntiles;
-  int kps = ((ntiles + s - 1) / s) * 64;
+  int kps = ((ntiles + s - 1) / s) * tile;
   s = (top_k + kps - 1) / kps;
   if (keys_per_split) *keys_per_split = kps;
   return s;
@@ -221,6 +222,7 @@ dsa_status check_index_inputs(const void* q_idx, dsa_dtype q_dtype, const float*
     return DSA_ERR_INVALID_ARG;
   }
   if (!aligned(q_idx, 16) || !aligned(k_cache, 16) || !aligned(head_w, 4)) return DSA_ERR_INVALID_ARG;
+  if (k_scale != nullptr && !aligned(k_scale, 16)) return DSA_ERR_INVALID_ARG;   // copied per page in bulk
   return DSA_OK;
 }
 

@@ -18,8 +18,10 @@ constexpr int kDimK = 576;
 constexpr int kDimV = 512;
 constexpr int kKvGroups = 5;
 
-// Bound of every wait inside a kernel (nanoseconds of %globaltimer).
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+// Bound of every wait inside a kernel, in SM clock cycles (about 1-3 s between the
+// lowest and the highest SM clock). The SM cycle counter is read instead of the
+// global timer because it is cheap enough to sit inside a polling loop.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // Layout of the 256-byte workspace header.
 struct WsHeader {
@@ -35,12 +37,6 @@ __device__ __forceinline__ void record_error(unsigned int* err, unsigned int cod
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -84,32 +80,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // raised `abort_flag`; the caller then records DSA_ERR_TIMEOUT and unwinds.
 __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
+  const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
+    if ((i & 255u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) return false;
+      if (clock64() - t0 > kWaitLimitCycles) return false;
     }
   }
 }
 
-// Warp-uniform bounded wait: every lane leaves with the same answer.
+// Warp-uniform bounded wait. Every lane tests the phase once (one round trip when it has
+// already completed, the common case); otherwise lane 0 polls alone and the other lanes
+// confirm afterwards, so a waiting warp issues few barrier operations.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  unsigned long long t0 = 0;
-  for (uint32_t i = 0;; ++i) {
-    const bool ok = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, ok)) return true;
-    if ((i & 63u) == 63u) {
-      int stop = 0;
-      if ((threadIdx.x & 31) == 0) {
-        const unsigned long long now = globaltimer();
-        if (t0 == 0) t0 = now;
-        stop = (*abort_flag != 0) || (now - t0 > kWaitLimitNs);
-      }
-      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
-    }
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) ok = wait_one(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait without the abort check, for draining in-flight copies on the way out.
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) break;
   }
+}
+
+// One lane of a converged warp (the lowest active one) returns true. tcgen05.mma and
+// tcgen05.commit are issued from such an elected lane of a converged warp: issuing them
+// from a lone divergent thread costs several times more per instruction.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies
@@ -228,6 +237,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 32 bit, 64 consecutive columns -> 64 registers per thread; waits for completion.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {

@@ -3,60 +3,86 @@
 //
 //   score[q, s] = k_scale[slot(s)] * sum_h (w[q,h] * q_scale[q,h]) * ReLU(<q8[q,h], k8[slot(s)]>)
 //
-// Design (sm_100a): one persistent CTA per SM walks a contiguous range of 128-token
-// tiles (two 64-token pages) of the paged key cache.
-//   warp 0  TMA producer: one 64 x 128 B box per page straight from the block table,
-//           128-byte swizzled, into an 8-deep ring; query tiles into a 2-slot ring.
-//   warp 1  tcgen05 issuer: D[128 tokens, 64*g heads] = K_tile x Q_group^T, fp8 x fp8
-//           (kind::f8f6f4) or bf16 x bf16 (kind::f16), fp32 in TMEM, 2 accumulators.
-//   warps 2-5  epilogue: one thread per token (its TMEM lane) applies ReLU, the head
-//           weights and the key scale, and writes the fp32 score row.
-// Decode (n_q = 1) loads a row's query once per row; chunked prefill streams groups
-// of up to 4 queries (N = 256) past every key tile.
+// Design (sm_100a): one persistent CTA per SM walks a contiguous range of 256-token
+// tiles (four 64-token pages) of the paged key cache.
+//   warp 0     TMA producer: one 64 x 128 B box per page, straight from the block table
+//              (fetched a batch ahead), 128-byte swizzled, into a 4-deep ring of 32 KB
+//              stages; query tiles into their own ring.
+//   warp 1     tcgen05 issuer: per 128-token half, D[128 tokens, 64*g heads] =
+//              K_half x Q_group^T, fp8 x fp8 (kind::f8f6f4) or bf16 x bf16 (kind::f16),
+//              fp32 in a ring of TMEM accumulators; MMAs come from an elected lane.
+//   warps 2-9  epilogue, two groups of four taking alternate accumulators: one thread
+//              per token (its TMEM lane) applies ReLU, the head weights and the key scale
+//              (loaded two tiles ahead) and writes the fp32 score.
+// Every synchronisation step costs a few hundred nanoseconds, so a tile carries 33 KB of
+// keys to keep that cost per byte low. Decode (n_q = 1) loads a row's query once per
+// row; chunked prefill streams groups of up to 4 queries (N = 256) past every key tile.
 #include "kernels.cuh"
 
 namespace dsa {
 
+constexpr int kTileTok = 256;
+constexpr int kPagesPerTile = kTileTok / kPage;
+constexpr int kQGroup = 4;
+constexpr int kBatch = 32 / kPagesPerTile;   // tiles whose block-table entries the producer fetches at once
+constexpr int kEpiWarps = 8;                 // two groups of four, alternating accumulators
+constexpr int kIdxThreads = 32 * (2 + kEpiWarps);
+constexpr uint32_t kIdxTmemCols = 512;       // accumulators of 64 * min(n_q, 4) columns each
+
 template <int KC>
 struct IdxCfg {
-  static constexpr int kStages = KC == 1 ? 8 : 2;
-  static constexpr int kBSlots = 2;
-  static constexpr int kAStage = KC * 16384;   // 128 tokens x 128 B per K-chunk
-  static constexpr int kBSlot = KC * 32768;    // 4 queries x 64 heads x 128 B per K-chunk
-  static constexpr int kWBytes = 4 * 2 * 256 * 4;  // per-warp double-buffered head weights
+  static constexpr int kChunk = kTileTok * 128;        // one 128-byte K-chunk of a tile
+  static constexpr int kStages = KC == 1 ? 4 : 2;
+  static constexpr int kBSlots = KC == 1 ? 2 : 1;
+  static constexpr int kAStage = KC * kChunk;          // 256 tokens x 128 B per K-chunk
+  static constexpr int kBSlot = KC * 32768;            // 4 queries x 64 heads x 128 B per K-chunk
+  static constexpr int kWBytes = kEpiWarps * 2 * 256 * 4;  // per-warp double-buffered head weights
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kAStage;
   static constexpr int kOffW = kOffB + kBSlots * kBSlot;
   static constexpr int kOffBar = kOffW + kWBytes;
-  static constexpr int kNumBars = 2 * kStages + 2 * kBSlots + 4 + 1;
+  static constexpr int kMaxAcc = 8;
+  static constexpr int kNumBars = 2 * kStages + 2 * kBSlots + 2 * kMaxAcc + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
 };
+static_assert(IdxCfg<1>::kSmem <= 232448 && IdxCfg<2>::kSmem <= 232448, "shared memory");
 
-constexpr int kTileTok = 128;
-constexpr int kQGroup = 4;
-constexpr uint32_t kIdxTmemCols = 512;  // 2 accumulators x 256 columns
-
-// Walks the CTA's contiguous range of global tile ids, yielding (row, tile-in-row).
+// Walks the CTA's contiguous range of global tile ids, yielding (row, tile-in-row) and
+// the row's clamped length. Row bounds and lengths live in registers and are reloaded
+// only when the walk crosses into the next row.
 struct TileWalker {
   const int32_t* prefix;
-  int b, gt, end;
-  __device__ void init(const int32_t* p, int B, int begin, int stop) {
-    prefix = p;
+  const int32_t* seq_lens;
+  int max_pages;
+  int b, gt, end, base, bound, len;
+  __device__ void init(const IndexerArgs& a, int begin, int stop) {
+    prefix = a.tile_prefix;
+    seq_lens = a.seq_lens;
+    max_pages = a.max_pages;
     gt = begin;
     end = stop;
-    int lo = 0, hi = B;  // largest b with prefix[b] <= begin
+    int lo = 0, hi = a.B;  // largest b with prefix[b] <= begin
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (prefix[mid] <= begin) lo = mid; else hi = mid;
     }
     b = lo;
+    base = prefix[b];
+    bound = prefix[b + 1];
+    len = row_len(seq_lens, b, max_pages);
   }
-  __device__ bool next(int& row, int& tile) {
+  __device__ bool next(int& row, int& tile, int& L) {
     if (gt >= end) return false;
-    while (gt >= prefix[b + 1]) ++b;
+    while (gt >= bound) {
+      ++b;
+      base = bound;
+      bound = prefix[b + 1];
+      len = row_len(seq_lens, b, max_pages);
+    }
     row = b;
-    tile = gt - prefix[b];
+    tile = gt - base;
+    L = len;
     ++gt;
     return true;
   }
@@ -72,15 +98,8 @@ __device__ __forceinline__ bool group_active(const IndexerArgs& a, int b, int g,
   return false;
 }
 
-__device__ __forceinline__ void bounded_drain(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) break;
-  }
-}
-
 template <int KC>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const IndexerArgs a) {
   using C = IdxCfg<KC>;
@@ -95,24 +114,27 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* b_full = a_empty + C::kStages;
   uint64_t* b_empty = b_full + C::kBSlots;
   uint64_t* acc_full = b_empty + C::kBSlots;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + C::kMaxAcc;
+  uint64_t* drain = acc_empty + C::kMaxAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // accumulator ring: 64 columns per query of a group; decode (n_q = 1) gets 8 of them
+  const int acc_cols = kHeads * min(a.n_q, kQGroup);
+  const int n_acc = min(C::kMaxAcc, static_cast<int>(kIdxTmemCols) / acc_cols);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&a_full[i], 1);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_empty[i], 1);   // the MMA commit
     }
     for (int i = 0; i < C::kBSlots; ++i) {
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::kMaxAcc; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
     }
@@ -137,30 +159,59 @@ __global__ void __launch_bounds__(192, 1)
 
   if (t_begin < t_end) {
     TileWalker walk;
-    walk.init(a.tile_prefix, a.B, t_begin, t_end);
+    walk.init(a, t_begin, t_end);
 
     if (warp == 0) {
-      // ------------------------------------------------------------ TMA producer
+      // ------------------------------------------------------------ TMA producer (whole warp)
+      // Lane 4i+p holds page p of batch tile i; the next batch's block-table loads are in
+      // flight while this one is issued. Lane 0 issues the page boxes and query tiles.
       if (lane == 0) {
         tma_prefetch_map(&tmap_k);
         tma_prefetch_map(&tmap_q);
-        int it = 0, bit = -1, cur_q0 = -1;
-        bool ok = true;
-        int b, t;
-        while (ok && walk.next(b, t)) {
-          const int L = row_len(a.seq_lens, b, a.max_pages);
-          const int npages = (L + kPage - 1) / kPage;
-          const int s = it % C::kStages;
-          if (!wait_one(&a_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          const int p0 = checked_page(a.block_table, b, 2 * t, a.max_pages, a.num_pages, a.err);
-          const bool has1 = 2 * t + 1 < npages;
-          const int p1 = has1 ? checked_page(a.block_table, b, 2 * t + 1, a.max_pages, a.num_pages, a.err) : 0;
-          mbar_arrive_expect_tx(&a_full[s], (has1 ? 2u : 1u) * KC * 8192u);
-          uint8_t* dst = sA + s * C::kAStage;
+      }
+      int it = 0, bit = -1, cur_q0 = -1;
+      bool ok = true;
+      auto load_batch = [&](int& n, int& my_b, int& my_t, int& my_L, int& my_page) {
+        n = 0;
+        my_b = my_t = my_L = 0;
+        for (; n < kBatch; ++n) {
+          int b, t, L;
+          if (!walk.next(b, t, L)) break;
+          if (lane / kPagesPerTile == n) { my_b = b; my_t = t; my_L = L; }
+        }
+        my_page = -1;
+        if (lane / kPagesPerTile < n) {
+          const int p = kPagesPerTile * my_t + (lane % kPagesPerTile);
+          if (p * kPage < my_L) my_page = checked_page(a.block_table, my_b, p, a.max_pages, a.num_pages, a.err);
+        }
+      };
+      int n, my_b, my_t, my_L, my_page;
+      load_batch(n, my_b, my_t, my_L, my_page);
+      while (ok && n > 0) {
+        int n2, nb, nt, nL, npg;
+        load_batch(n2, nb, nt, nL, npg);
+        for (int i = 0; i < n; ++i) {
+          const int src = kPagesPerTile * i;
+          const int b = __shfl_sync(0xffffffffu, my_b, src);
+          const int t = __shfl_sync(0xffffffffu, my_t, src);
+          const int L = __shfl_sync(0xffffffffu, my_L, src);
+          int pages[kPagesPerTile];
 #pragma unroll
-          for (int kc = 0; kc < KC; ++kc) {
-            tma_load_2d(dst + kc * 16384, &tmap_k, kc * 64, p0 * kPage, &a_full[s]);
-            if (has1) tma_load_2d(dst + kc * 16384 + 8192, &tmap_k, kc * 64, p1 * kPage, &a_full[s]);
+          for (int p = 0; p < kPagesPerTile; ++p) pages[p] = __shfl_sync(0xffffffffu, my_page, src + p);
+          const int s = it % C::kStages;
+          if (!wait_warp(&a_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (lane == 0) {
+            uint32_t npages = 0;
+#pragma unroll
+            for (int p = 0; p < kPagesPerTile; ++p) npages += pages[p] >= 0 ? 1u : 0u;
+            mbar_arrive_expect_tx(&a_full[s], npages * KC * 8192u);
+            uint8_t* dst = sA + s * C::kAStage;
+#pragma unroll
+            for (int p = 0; p < kPagesPerTile; ++p)
+              if (pages[p] >= 0)
+#pragma unroll
+                for (int kc = 0; kc < KC; ++kc)
+                  tma_load_2d(dst + kc * C::kChunk + p * 8192, &tmap_k, kc * 64, pages[p] * kPage, &a_full[s]);
           }
           ++it;
           const int tok0 = t * kTileTok;
@@ -171,136 +222,189 @@ __global__ void __launch_bounds__(192, 1)
             const int nqg = min(kQGroup, a.n_q - g * kQGroup);
             ++bit;
             const int bs = bit % C::kBSlots;
-            if (!wait_one(&b_empty[bs], ((bit / C::kBSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&b_full[bs], static_cast<uint32_t>(nqg) * KC * 8192u);
-            for (int j = 0; j < nqg; ++j)
+            if (!wait_warp(&b_empty[bs], ((bit / C::kBSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&b_full[bs], static_cast<uint32_t>(nqg) * KC * 8192u);
+              for (int j = 0; j < nqg; ++j)
 #pragma unroll
-              for (int kc = 0; kc < KC; ++kc)
-                tma_load_2d(sB + bs * C::kBSlot + kc * 32768 + j * 8192, &tmap_q, kc * 64, (q0 + j) * kHeads,
-                            &b_full[bs]);
+                for (int kc = 0; kc < KC; ++kc)
+                  tma_load_2d(sB + bs * C::kBSlot + kc * 32768 + j * 8192, &tmap_q, kc * 64, (q0 + j) * kHeads,
+                              &b_full[bs]);
+            }
             cur_q0 = q0;
           }
+          if (!ok) break;
         }
-        if (!ok) {
-          record_error(a.err, DSA_ERR_TIMEOUT, 1);
-          *abort_flag = 1;
-          for (int i = max(0, it - C::kStages); i < it; ++i) bounded_drain(&a_full[i % C::kStages], (i / C::kStages) & 1);
-          for (int i = max(0, bit - C::kBSlots + 1); i <= bit; ++i)
-            bounded_drain(&b_full[i % C::kBSlots], (i / C::kBSlots) & 1);
-        }
+        n = n2; my_b = nb; my_t = nt; my_L = nL; my_page = npg;
+      }
+      if (!ok && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 1);
+        *abort_flag = 1;
+      }
+      if (lane == 0) {
+        for (int i = max(0, it - C::kStages); i < it; ++i) wait_drain(&a_full[i % C::kStages], (i / C::kStages) & 1);
+        for (int i = max(0, bit - C::kBSlots + 1); i <= bit; ++i)
+          wait_drain(&b_full[i % C::kBSlots], (i / C::kBSlots) & 1);
       }
       __syncwarp();
     } else if (warp == 1) {
-      // ------------------------------------------------------------ tcgen05 issuer
-      if (lane == 0) {
-        const uint32_t fmt = KC == 1 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
-        int it = 0, bit = -1, cur_q0 = -1, acc_it = 0;
-        bool ok = true;
-        int b, t;
-        while (ok && walk.next(b, t)) {
-          const int L = row_len(a.seq_lens, b, a.max_pages);
-          const int s = it % C::kStages;
-          if (!wait_one(&a_full[s], (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const int tok0 = t * kTileTok;
-          const uint32_t a_base = smem_u32(sA + s * C::kAStage);
-          for (int g = 0; g < ngroups && ok; ++g) {
-            if (!group_active(a, b, g, tok0, L)) continue;
-            const int q0 = b * a.n_q + g * kQGroup;
-            const int nqg = min(kQGroup, a.n_q - g * kQGroup);
-            if (q0 != cur_q0) {
-              if (bit >= 0) tc_commit(&b_empty[bit % C::kBSlots]);
-              ++bit;
-              if (!wait_one(&b_full[bit % C::kBSlots], (bit / C::kBSlots) & 1, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              cur_q0 = q0;
-            }
-            const int ab = acc_it & 1;
-            if (!wait_one(&acc_empty[ab], ((acc_it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d = tmem + static_cast<uint32_t>(ab * 256);
-            const uint32_t idesc = idesc_make(fmt, fmt, false, false, 128, kHeads * nqg);
-            const uint32_t b_base = smem_u32(sB + (bit % C::kBSlots) * C::kBSlot);
-#pragma unroll
-            for (int kc = 0; kc < KC; ++kc)
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = sdesc_sw128(a_base + kc * 16384 + ks * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(b_base + kc * 32768 + ks * 32, 16, 1024);
-                if (KC == 1) mma_f8(d, ad, bd, idesc, (kc | ks) != 0);
-                else mma_f16(d, ad, bd, idesc, (kc | ks) != 0);
-              }
-            tc_commit(&acc_full[ab]);
-            ++acc_it;
-          }
-          if (!ok) break;
-          tc_commit(&a_empty[s]);
-          ++it;
-        }
-        if (!ok) {
-          record_error(a.err, DSA_ERR_TIMEOUT, 2);
-          *abort_flag = 1;
-        }
-        // every MMA this thread issued has finished before the CTA frees TMEM
-        tc_commit(drain);
-        bounded_drain(drain, 0);
-      }
-      __syncwarp();
-    } else {
-      // ------------------------------------------------------------ epilogue (warps 2..5)
-      const int quarter = warp & 3;            // TMEM lanes [32*quarter, 32*quarter + 32)
-      const int row_in_tile = quarter * 32 + lane;
-      float* wmine = sW + (warp - 2) * 512;    // two 256-entry buffers per warp
-      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      int acc_it = 0, cur_q0 = -1, wb = 1;
+      // ------------------------------------------------------------ tcgen05 issuer (whole warp)
+      // Descriptors are formed once and advanced by constants (the start address field is
+      // address / 16); the MMAs and their commits come from one elected lane.
+      const uint32_t fmt = KC == 1 ? 0u : 1u;  // e4m3 (kind::f8f6f4) or bf16 (kind::f16)
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+      int it = 0, bit = -1, cur_q0 = -1, unit = 0;
       bool ok = true;
-      int b, t;
-      while (ok && walk.next(b, t)) {
-        const int L = row_len(a.seq_lens, b, a.max_pages);
+      int b, t, L;
+      while (ok && walk.next(b, t, L)) {
+        const int s = it % C::kStages;
+        if (!wait_warp(&a_full[s], (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
         const int tok0 = t * kTileTok;
-        const int tok = tok0 + row_in_tile;
-        float kscale = 1.0f;
-        if (a.k_scale != nullptr && tok < L) {
-          const int pg = checked_page(a.block_table, b, tok >> 6, a.max_pages, a.num_pages, a.err);
-          kscale = a.k_scale[static_cast<int64_t>(pg) * kPage + (tok & 63)];
-        }
-        for (int g = 0; g < ngroups; ++g) {
+        const uint64_t ad = a_desc0 + static_cast<uint64_t>((s * C::kAStage) >> 4);
+        for (int g = 0; g < ngroups && ok; ++g) {
           if (!group_active(a, b, g, tok0, L)) continue;
           const int q0 = b * a.n_q + g * kQGroup;
           const int nqg = min(kQGroup, a.n_q - g * kQGroup);
           if (q0 != cur_q0) {
-            wb ^= 1;
-            __syncwarp();
-            for (int i = lane; i < nqg * kHeads; i += 32) {
-              float w = a.head_w[static_cast<int64_t>(q0) * kHeads + i];
-              if (a.q_scale != nullptr) w *= a.q_scale[static_cast<int64_t>(q0) * kHeads + i];
-              wmine[wb * 256 + i] = w;
+            if (bit >= 0) {
+              if (elect_one()) tc_commit(&b_empty[bit % C::kBSlots]);
+              __syncwarp();
             }
-            __syncwarp();
+            ++bit;
+            if (!wait_warp(&b_full[bit % C::kBSlots], (bit / C::kBSlots) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
             cur_q0 = q0;
           }
-          const int ab = acc_it & 1;
-          if (!wait_warp(&acc_full[ab], (acc_it >> 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          for (int j = 0; j < nqg; ++j) {
-            float acc[32];
-            float sc = 0.0f;
-            const float* wq = wmine + wb * 256 + j * kHeads;
+          const uint32_t idesc = idesc_make(fmt, fmt, false, false, 128, kHeads * nqg);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>(((bit % C::kBSlots) * C::kBSlot) >> 4);
+          for (int h2 = 0; h2 < 2; ++h2, ++unit) {
+            const int ab = unit % n_acc;
+            if (!wait_warp(&acc_empty[ab], ((unit / n_acc) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d = tmem + static_cast<uint32_t>(ab * acc_cols);
+            if (elect_one()) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              tmem_ld32(lane_addr + static_cast<uint32_t>(ab * 256 + j * kHeads + half * 32), acc);
+              for (int kc = 0; kc < KC; ++kc)
 #pragma unroll
-              for (int h = 0; h < 32; ++h) sc = fmaf(wq[half * 32 + h], fmaxf(acc[h], 0.0f), sc);
+                for (int ks = 0; ks < 4; ++ks) {
+                  const uint64_t ao = ad + static_cast<uint64_t>((kc * C::kChunk + h2 * 16384 + ks * 32) >> 4);
+                  const uint64_t bo = bd + static_cast<uint64_t>((kc * 32768 + ks * 32) >> 4);
+                  if (KC == 1) mma_f8(d, ao, bo, idesc, (kc | ks) != 0);
+                  else mma_f16(d, ao, bo, idesc, (kc | ks) != 0);
+                }
+              tc_commit(&acc_full[ab]);
             }
-            const int q = q0 + j;
-            int vis = query_vis(a.q_pos, q, L);
-            if (vis > a.L_max) vis = static_cast<int>(a.L_max);
-            if (tok < vis) a.scores[static_cast<int64_t>(q) * a.L_max + tok] = sc * kscale;
+            __syncwarp();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          ++acc_it;
+        }
+        if (!ok) break;
+        if (elect_one()) tc_commit(&a_empty[s]);
+        __syncwarp();
+        ++it;
+      }
+      if (!ok && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 2);
+        *abort_flag = 1;
+      }
+      // every MMA this warp issued has finished before the CTA frees TMEM
+      if (elect_one()) {
+        tc_commit(drain);
+        wait_drain(drain, 0);
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------------ epilogue (warps 2..9)
+      // Two groups of four warps take alternate accumulator units (a unit = a 128-token half
+      // of a tile for one query group); in a group, warp w reads TMEM lanes
+      // [32*(w%4), 32*(w%4)+32), one token per thread. Each thread loads the key scales of
+      // its two tokens of a tile two tiles ahead, from block-table entries loaded four tiles
+      // ahead, so neither load stalls the tile it is used in.
+      const int eg = (warp - 2) >> 2;
+      const int quarter = warp & 3;
+      const int row_in_half = quarter * 32 + lane;
+      float* wmine = sW + (warp - 2) * 512;    // two 256-entry buffers per warp
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+      int unit = 0, cur_q0 = -1, wb = 1;
+      bool ok = true;
+      TileWalker w2 = walk, w4 = walk;
+      // page of this thread's token in half h of the next tile of walker w (-1 past the end)
+      auto tile_pages = [&](TileWalker& w, int& p0, int& p1, int& o) {
+        int bb, tt, LL;
+        p0 = p1 = -1;
+        o = row_in_half & 63;
+        if (!w.next(bb, tt, LL)) return;
+        if (a.k_scale == nullptr) return;
+        const int tk0 = tt * kTileTok + row_in_half;
+        if (tk0 < LL) p0 = checked_page(a.block_table, bb, tk0 >> 6, a.max_pages, a.num_pages, a.err);
+        if (tk0 + 128 < LL) p1 = checked_page(a.block_table, bb, (tk0 + 128) >> 6, a.max_pages, a.num_pages, a.err);
+      };
+      auto load_scale = [&](int page, int o) {
+        return page >= 0 ? __ldg(a.k_scale + static_cast<int64_t>(page) * kPage + o) : 1.0f;
+      };
+      int pa0, pa1, pb0, pb1, pc0, pc1, pd0, pd1, off;
+      tile_pages(w2, pa0, pa1, off);
+      tile_pages(w2, pb0, pb1, off);
+      float ks00 = load_scale(pa0, off), ks01 = load_scale(pa1, off);   // tile +0
+      float ks10 = load_scale(pb0, off), ks11 = load_scale(pb1, off);   // tile +1
+      w4 = w2;
+      tile_pages(w4, pc0, pc1, off);                                    // tile +2
+      tile_pages(w4, pd0, pd1, off);                                    // tile +3
+      int b, t, L;
+      while (ok && walk.next(b, t, L)) {
+        const float kscale[2] = {ks00, ks01};
+        ks00 = ks10; ks01 = ks11;
+        ks10 = load_scale(pc0, off); ks11 = load_scale(pc1, off);
+        pc0 = pd0; pc1 = pd1;
+        tile_pages(w4, pd0, pd1, off);
+        const int tok0 = t * kTileTok;
+        for (int g = 0; g < ngroups && ok; ++g) {
+          if (!group_active(a, b, g, tok0, L)) continue;
+          const int q0 = b * a.n_q + g * kQGroup;
+          const int nqg = min(kQGroup, a.n_q - g * kQGroup);
+          for (int h2 = 0; h2 < 2; ++h2, ++unit) {
+            if ((unit & 1) != eg) continue;
+            if (q0 != cur_q0) {
+              wb ^= 1;
+              __syncwarp();
+              for (int i = lane; i < nqg * kHeads; i += 32) {
+                float w = a.head_w[static_cast<int64_t>(q0) * kHeads + i];
+                if (a.q_scale != nullptr) w *= a.q_scale[static_cast<int64_t>(q0) * kHeads + i];
+                wmine[wb * 256 + i] = w;
+              }
+              __syncwarp();
+              cur_q0 = q0;
+            }
+            const int ab = unit % n_acc;
+            if (!wait_warp(&acc_full[ab], (unit / n_acc) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const int tok = tok0 + h2 * 128 + row_in_half;
+            for (int j = 0; j < nqg; ++j) {
+              float acc[64];
+              tmem_ld64(lane_addr + static_cast<uint32_t>(ab * acc_cols + j * kHeads), acc);
+              const float4* wq = reinterpret_cast<const float4*>(wmine + wb * 256 + j * kHeads);
+              float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent chains
+#pragma unroll
+              for (int h4 = 0; h4 < 16; ++h4) {
+                const float4 w = wq[h4];
+                float* pp = part + 4 * (h4 & 1);
+                pp[0] = fmaf(w.x, fmaxf(acc[4 * h4 + 0], 0.0f), pp[0]);
+                pp[1] = fmaf(w.y, fmaxf(acc[4 * h4 + 1], 0.0f), pp[1]);
+                pp[2] = fmaf(w.z, fmaxf(acc[4 * h4 + 2], 0.0f), pp[2]);
+                pp[3] = fmaf(w.w, fmaxf(acc[4 * h4 + 3], 0.0f), pp[3]);
+              }
+              const float sc =
+                  ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+              const int q = q0 + j;
+              int vis = query_vis(a.q_pos, q, L);
+              if (vis > a.L_max) vis = static_cast<int>(a.L_max);
+              if (tok < vis) a.scores[static_cast<int64_t>(q) * a.L_max + tok] = sc * kscale[h2];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          }
         }
       }
       if (!ok && lane == 0) {
@@ -364,10 +468,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, con
   }
 }
 
-template __global__ void indexer_kernel<1>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                                           const IndexerArgs);
-template __global__ void indexer_kernel<2>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                                           const IndexerArgs);
+
 
 cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches) {
@@ -382,7 +483,7 @@ static cudaError_t launch_indexer_kc(const CUtensorMap& tk, const CUtensorMap& t
   constexpr int smem = IdxCfg<KC>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(indexer_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  indexer_kernel<KC><<<grid, 192, smem, stream>>>(tk, tq, a);
+  indexer_kernel<KC><<<grid, kIdxThreads, smem, stream>>>(tk, tq, a);
   return cudaGetLastError();
 }
 

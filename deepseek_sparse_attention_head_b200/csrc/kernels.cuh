@@ -40,7 +40,7 @@ struct MlaArgs {
   int Bq;
   int top_k;
   int nsplit;
-  int keys_per_split;   // multiple of 64
+  int keys_per_split;   // multiple of mla_tile_keys()
   const uint8_t* kv;    // [num_slots, 576] fp8 codes or bf16 values
   const float* kv_scale;
   int64_t num_slots;
@@ -65,5 +65,6 @@ cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* blo
                            int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,
                            cudaStream_t stream, int* launches);
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
+int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
 }  // namespace dsa

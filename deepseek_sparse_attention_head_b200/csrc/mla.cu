@@ -5,16 +5,23 @@
 //
 // (576 = 512 latent + 64 rope columns; "Show HN: colibri", features.)
 //
-// Design (sm_100a): grid = (query, split); each CTA walks 64-row tiles of its share of
-// the index list.
-//   * fp8 rows (576 B) are fetched with one bulk async copy each into a 2-deep ring,
-//     then dequantised (code x per-group scale -> bf16) into a 128-byte-swizzled tile
-//     that serves both as the K operand of QK and the (MN-major) V operand of PV.
-//   * QK:  S[heads, keys] = Q[64 (+64 unused rows), 576] x KV^T    (tcgen05 kind::f16, M=128)
-//   * softmax per head (one thread per head, row in TMEM), lazily rescaled: the
-//     running max only moves when a tile's max exceeds it by more than 8 (log2 units).
-//   * PV:  O^T[512 dims, 64 heads] += V^T x P^T                    (4 x M=128, N=64)
-// Splits write (m, l, o) partials; a combine kernel merges them with log-sum-exp.
+// Design (sm_100a): grid = (query, split); a CTA walks 32-row tiles of its share of
+// the index list with warp-specialised, double-buffered stages:
+//   warp 1    producer: the tile's slot ids, one 576-byte bulk async copy per fp8 row
+//             into a 3-deep ring, and the row's five scales folded into an exact
+//             power-of-two row exponent E_j plus five fp16 multipliers s_g / 2^E_j;
+//   warps 2-3 dequantisers: fp8 code -> fp16 (exact) x multiplier -> fp16 tile,
+//             128-byte swizzled; the tile is the K operand of QK (K-major) and the
+//             V operand of PV (MN-major) at once;
+//   warp 0    tcgen05 issuer:  S = Q' K'^T (M=128, rows 64..127 unused, N=32),
+//             O^T += V'^T P'^T (4 x M=128, N=64); fp32 accumulators in TMEM;
+//   warps 4-5 softmax, one thread per head (its TMEM lane): running max with lazy
+//             rescaling (only when a tile's max exceeds it by more than 8 in log2
+//             units), exact fp32 normaliser, fp16 weights P' = p * 2^(E_j - E_ref);
+//   warps 4-7 the rare O rescale and the output epilogue (all 128 TMEM lanes).
+// Q is staged once per CTA and rescaled per head by a power of two into fp16. With
+// a bf16 cache the same pipeline runs in bf16 without any rescaling.
+// Splits write (m, l, o) partials that mla_combine_kernel merges by log-sum-exp.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -23,46 +30,77 @@
 
 namespace dsa {
 
-constexpr int kMlaTile = 64;
-constexpr int kMlaThreads = 128;
-constexpr uint32_t kMlaTmemCols = 512;   // S: cols [0,64); O^T: cols [64, 320)
-constexpr int kOffQ = 0;                 // 9 x 8 KB, K-major SW128
-constexpr int kOffKV = 73728;            // 9 x 8 KB, K-major SW128 (rows = keys)
-constexpr int kOffP = 147456;            // 64 heads x 128 B
-constexpr int kOffStage = 155648;        // 2 x 64 x 576 B fp8 staging
-constexpr int kStageBytes = kMlaTile * kDimK;
-constexpr int kOffIdx = kOffStage + 2 * kStageBytes;   // 2 x 64 int32
-constexpr int kOffAlpha = kOffIdx + 512;               // 64 f32
-constexpr int kOffInvL = kOffAlpha + 256;              // 64 f32
-constexpr int kOffMisc = kOffInvL + 256;               // vmask (u64), tmem holder, abort
-constexpr int kOffBars = kOffMisc + 64;                // q_full, stage_full[2], s_done, o_done
-constexpr int kMlaSmem = kOffBars + 64 + 1024;
+constexpr int kMlaTile = 32;
+constexpr int kMlaThreads = 256;
+constexpr int kMlaStages = 3;
+constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,64); O^T: cols [64, 320)
+constexpr int kRowBytes = kDimK;              // fp8 row
+constexpr int kStageRows = kMlaTile * kRowBytes;
+constexpr int kNoExp = -100000;               // "no valid row seen yet"
 
-__device__ __forceinline__ void store_swizzled(uint8_t* tile, int row, int chunk16, uint4 v) {
-  // row-major [rows][128 B] block of one 64-element K chunk, 16-byte unit swizzled by row % 8
-  *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk16 ^ (row & 7)) << 4)) = v;
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr int kOffQ = 0;                                        // 9 x [64 x 128 B]
+constexpr int kOffStage = kOffQ + 9 * 8192;                     // 3 x [32 x 576 B]
+constexpr int kOffStageMeta = kOffStage + kMlaStages * kStageRows;
+constexpr int kStageMetaBytes = 1024;                           // mult[32][5] u32, E[32], slot[32]
+constexpr int kOffKV = kOffStageMeta + kMlaStages * kStageMetaBytes;   // 2 x 9 x [32 x 128 B]
+constexpr int kKVChunk = kMlaTile * 128;
+constexpr int kKVBytes = 9 * kKVChunk;
+constexpr int kOffP = kOffKV + 2 * kKVBytes;                    // [64 heads x 128 B]; tile parity picks the half
+constexpr int kOffKVMeta = kOffP + 8192;                        // 2 x (E[32], vmask)
+constexpr int kOffHead = kOffKVMeta + 512;                      // cq[64], alpha[64], outscale[64]
+constexpr int kOffIdxList = kOffHead + 768;                     // the split's slot list (<= 2048 entries)
+constexpr int kIdxListCap = 2048;
+constexpr int kOffBars = kOffIdxList + kIdxListCap * 4;
+constexpr int kOffMisc = kOffBars + 256;
+constexpr int kMlaSmem = kOffMisc + 64 + 1024;
+
+static_assert(kOffKV % 1024 == 0 && kOffP % 1024 == 0 && kOffStage % 16 == 0, "alignment");
+static_assert(kMlaSmem <= 232448, "shared memory");
+
+// OR / AND over the 128 threads of warps 4..7 (named barrier 1).
+__device__ __forceinline__ int group_or(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return static_cast<int>(r);
+}
+__device__ __forceinline__ int group_and(int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return static_cast<int>(r);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&t);
+__device__ __forceinline__ uint32_t swz(int row, int unit) {  // 128-byte swizzle inside an 8-row atom
+  return static_cast<uint32_t>(row * 128 + ((unit ^ (row & 7)) << 4));
 }
 
-// Four E4M3 codes (one 32-bit word) times `sc` -> two bf16x2 words.
-__device__ __forceinline__ void dequant4(uint32_t w, float sc, uint32_t& o0, uint32_t& o1) {
-  const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
-  const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-  const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-  o0 = pack_bf16x2(f01.x * sc, f01.y * sc);
-  o1 = pack_bf16x2(f23.x * sc, f23.y * sc);
+__device__ __forceinline__ int float_exponent(float s) {  // floor(log2 s) for positive normal s
+  return static_cast<int>((__float_as_uint(s) >> 23) & 0xFF) - 127;
 }
 
-__device__ __forceinline__ void bounded_wait(uint64_t* bar, uint32_t parity) {
-  const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) break;
-  }
+__device__ __forceinline__ float exp2i(int e) {  // exact 2^e, clamped to the normal fp32 range
+  e = e < -126 ? -126 : (e > 127 ? 127 : e);
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+// Four E4M3 codes -> four fp16 (exact) times the fp16 multiplier pair m2.
+__device__ __forceinline__ void dequant4_f16(uint32_t w, __half2 m2, uint32_t& o0, uint32_t& o1) {
+  const __half2_raw r01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw r23 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  __half2 h01 = __hmul2(*reinterpret_cast<const __half2*>(&r01), m2);
+  __half2 h23 = __hmul2(*reinterpret_cast<const __half2*>(&r23), m2);
+  o0 = *reinterpret_cast<uint32_t*>(&h01);
+  o1 = *reinterpret_cast<uint32_t*>(&h23);
 }
 
 template <bool FP8>
@@ -71,21 +109,27 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
+  uint8_t* sStage = smem + kOffStage;
+  uint8_t* sStageMeta = smem + kOffStageMeta;
   uint8_t* sKV = smem + kOffKV;
   uint8_t* sP = smem + kOffP;
-  uint8_t* sStage = smem + kOffStage;
-  int32_t* sIdx = reinterpret_cast<int32_t*>(smem + kOffIdx);
-  float* sAlpha = reinterpret_cast<float*>(smem + kOffAlpha);
-  float* sInvL = reinterpret_cast<float*>(smem + kOffInvL);
-  unsigned long long* sVmask = reinterpret_cast<unsigned long long*>(smem + kOffMisc);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 12);
+  int32_t* sKVMeta = reinterpret_cast<int32_t*>(smem + kOffKVMeta);
+  float* sCq = reinterpret_cast<float*>(smem + kOffHead);
+  float* sAlpha = sCq + 64;
+  float* sOutScale = sCq + 128;
+  int32_t* sIdxList = reinterpret_cast<int32_t*>(smem + kOffIdxList);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
-  uint64_t* q_full = bars;
-  uint64_t* stage_full = bars + 1;  // [2]
-  uint64_t* s_done = bars + 3;
-  uint64_t* o_done = bars + 4;
-  uint64_t* drain = bars + 5;
+  uint64_t* q_full = bars + 0;
+  uint64_t* stage_full = bars + 1;    // [3]
+  uint64_t* stage_empty = bars + 4;   // [3]
+  uint64_t* kv_full = bars + 7;       // [2]
+  uint64_t* s_full = bars + 9;        // [2]
+  uint64_t* s_empty = bars + 11;      // [2]
+  uint64_t* p_full = bars + 13;       // [2]
+  uint64_t* pv_done = bars + 15;      // [2]
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -100,10 +144,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&stage_full[0], 1);
-    mbar_init(&stage_full[1], 1);
-    mbar_init(s_done, 1);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < kMlaStages; ++i) {
+      mbar_init(&stage_full[i], 1);
+      mbar_init(&stage_empty[i], 2);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 2);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 2);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -116,278 +167,453 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_S = tmem;
   const uint32_t tmem_O = tmem + 64;
 
-  // Reads tile T's slot list into sIdx[st] (invalid -> -1) and, for fp8, starts one
-  // bulk copy per valid row into staging buffer st. Executed by warp 3.
-  auto issue_tile = [&](int T, int st) {
-    int32_t* idx = sIdx + st * kMlaTile;
-    int slots[2];
-    unsigned valid = 0;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int j = lane + 32 * r;
-      const int k = k0 + T * kMlaTile + j;
-      int slot = k < k1 ? phys[k] : -1;
+  // the split's slot list, staged once (invalid entries become -1)
+  const bool list_in_smem = nkeys <= kIdxListCap;
+  if (list_in_smem) {
+    for (int i = tid; i < ntiles * kMlaTile; i += kMlaThreads) {
+      int slot = i < nkeys ? phys[k0 + i] : -1;
       if (slot < -1 || slot >= a.num_slots) {
         record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(slot));
         slot = -1;
       }
-      slots[r] = slot;
-      idx[j] = slot;
-      valid += slot >= 0 ? 1u : 0u;
+      sIdxList[i] = slot;
     }
-    if (FP8) {
-      unsigned nvalid = valid;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, off);
-      if (lane == 0) mbar_arrive_expect_tx(&stage_full[st], nvalid * kDimK);
-      __syncwarp();
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int j = lane + 32 * r;
-        if (slots[r] >= 0)
-          bulk_load(sStage + st * kStageBytes + j * kDimK, a.kv + static_cast<int64_t>(slots[r]) * kDimK, kDimK,
-                    &stage_full[st]);
-      }
-    }
-    __syncwarp();
-  };
-
-  if (tid == 0 && ntiles > 0) {
-    tma_prefetch_map(&tmap_q);
-    mbar_arrive_expect_tx(q_full, 9u * 8192u);
-#pragma unroll 1
-    for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
-  }
-  if (warp == 3) {
-    if (ntiles > 0) issue_tile(0, 0);
-    if (ntiles > 1) issue_tile(1, 1);
   }
 
-  float m_run = -INFINITY, l_run = 0.0f;   // per head (threads 0..63)
+  // ---------------------------------------------------------------- Q: load, rescale per head
   bool ok = true;
-  int issued = min(ntiles, 2);             // tiles whose rows have been requested
-  int T = 0;
-  if (ntiles > 0) ok = wait_warp(q_full, 0, abort_flag);
-  __syncthreads();
-
-  const uint32_t idesc_qk = idesc_make(1, 1, false, false, 128, 64);
-  const uint32_t idesc_pv = idesc_make(1, 1, true, false, 128, 64);
-
-#pragma unroll 1
-  for (; T < ntiles; ++T) {
-    const int st = T & 1;
-    if (FP8) {
-      const bool got = wait_warp(&stage_full[st], (T >> 1) & 1, abort_flag);
-      ok = __syncthreads_and(got && ok);
-      if (!ok) break;
+  if (ntiles > 0) {
+    if (tid == 0) {
+      tma_prefetch_map(&tmap_q);
+      mbar_arrive_expect_tx(q_full, 9u * 8192u);
+      for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
     }
-    // ---- dequantise the tile into the swizzled bf16 KV tile
-    const int32_t* idx = sIdx + st * kMlaTile;
-    if (FP8) {
-      const uint8_t* stage = sStage + st * kStageBytes;
-#pragma unroll 2
-      for (int c = tid; c < kMlaTile * 36; c += kMlaThreads) {
-        const int j = c / 36, cc = c - j * 36;
-        const int slot = idx[j];
-        uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-        if (slot >= 0) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(stage + j * kDimK + cc * 16);
-          const float sc = a.kv_scale[static_cast<int64_t>(slot) * kKvGroups + (cc >> 3)];
-          dequant4(raw.x, sc, o0.x, o0.y);
-          dequant4(raw.y, sc, o0.z, o0.w);
-          dequant4(raw.z, sc, o1.x, o1.y);
-          dequant4(raw.w, sc, o1.z, o1.w);
+    ok = wait_warp(q_full, 0, abort_flag);
+    const int h = tid >> 2, part = tid & 3;   // 4 threads per head, 18 of its 72 16-byte units each
+    int F = 0;
+    if (FP8 && ok) {
+      float mx = 0.0f;
+      for (int u = part * 18; u < part * 18 + 18; ++u) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
         }
-        uint8_t* blk = sKV + (cc >> 2) * 8192;
-        store_swizzled(blk, j, (cc & 3) * 2, o0);
-        store_swizzled(blk, j, (cc & 3) * 2 + 1, o1);
       }
-    } else {
-      for (int c = tid; c < kMlaTile * 72; c += kMlaThreads) {
-        const int j = c / 72, cc = c - j * 72;
-        const int slot = idx[j];
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (slot >= 0) v = *reinterpret_cast<const uint4*>(a.kv + static_cast<int64_t>(slot) * (2 * kDimK) + cc * 16);
-        store_swizzled(sKV + (cc >> 3) * 8192, j, cc & 7, v);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      F = mx > 0.0f ? float_exponent(mx) : 0;
+      const float inv = exp2i(-F);
+      for (int u = part * 18; u < part * 18 + 18; ++u) {
+        uint4* p = reinterpret_cast<uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
+        const uint4 v = *p;
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+          __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
+          w[i] = *reinterpret_cast<uint32_t*>(&hh);
+        }
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
-    if (warp == 0) {
-      const unsigned lo = __ballot_sync(0xffffffffu, idx[lane] >= 0);
-      const unsigned hi = __ballot_sync(0xffffffffu, idx[32 + lane] >= 0);
-      if (lane == 0) *sVmask = (static_cast<unsigned long long>(hi) << 32) | lo;
-    }
+    if (part == 0) sCq[h] = a.scale_log2 * exp2i(F);
     fence_proxy_async_smem();
-    __syncthreads();
+  }
+  ok = __syncthreads_and(ok) != 0;
 
-    // ---- refill this staging buffer; issue QK
-    if (warp == 3 && T + 2 < ntiles) issue_tile(T + 2, st);
-    if (T + 2 < ntiles) issued = T + 3;
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t q_base = smem_u32(sQ), kv_base = smem_u32(sKV);
-#pragma unroll 1
-      for (int kc = 0; kc < 9; ++kc)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem_S, sdesc_sw128(q_base + kc * 8192 + ks * 32, 16, 1024),
-                  sdesc_sw128(kv_base + kc * 8192 + ks * 32, 16, 1024), idesc_qk, (kc | ks) != 0);
-      tc_commit(s_done);
-    }
+  // fp16 operands for an fp8 cache, bf16 for a bf16 cache
+  const uint32_t fmt = FP8 ? 0u : 1u;
+  const uint32_t idesc_qk = idesc_make(fmt, fmt, false, false, 128, kMlaTile);
+  const uint32_t idesc_pv = idesc_make(fmt, fmt, true, false, 128, 64);
 
-    // ---- softmax: thread h < 64 owns head h (TMEM lane h)
-    int need_rescale = 0;
-    bool got = true;
-    if (warp < 2) {
-      got = wait_warp(s_done, T & 1, abort_flag);
-      if (got) {
+  if (ok && ntiles > 0) {
+    if (warp == 0) {
+      // ------------------------------------------------------------ tcgen05 issuer (whole warp)
+      // Descriptors are formed once and advanced by constants; MMAs and commits come from
+      // one elected lane of the converged warp.
+      bool good = true;
+      const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);                 // K-major view
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);            // MN-major view
+      const uint64_t p_desc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      auto issue_pv = [&](int T) {
+        const int b = T & 1;
+        if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        const unsigned long long vm = *sVmask;
-        const int h = tid;
-        float z[64];
-        {
-          float tmp[32];
-          tmem_ld32(tmem_S + (static_cast<uint32_t>(warp * 32) << 16), tmp);
+        const uint64_t vb = v_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
+        const uint64_t pb = p_desc0 + static_cast<uint64_t>((b * 64) >> 4);
+        if (elect_one()) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = tmp[i];
-          tmem_ld32(tmem_S + (static_cast<uint32_t>(warp * 32) << 16) + 32, tmp);
+          for (int d = 0; d < 4; ++d)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) z[32 + i] = tmp[i];
+            for (int ks = 0; ks < 2; ++ks)
+              mma_f16(tmem_O + d * 64, vb + static_cast<uint64_t>(((2 * d) * kKVChunk + ks * 2048) >> 4),
+                      pb + static_cast<uint64_t>((ks * 32) >> 4), idesc_pv, (T > 0 || ks > 0) ? 1u : 0u);
+          tc_commit(&pv_done[b]);
         }
-        float mt = -INFINITY;
+        __syncwarp();
+        return true;
+      };
+      for (int T = 0; T < ntiles; ++T) {
+        const int b = T & 1;
+        if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag)) { good = false; break; }
+        if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
+        tc_fence_after();
+        const uint64_t kb = kv_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
+        if (elect_one()) {
+#pragma unroll 3
+          for (int kc = 0; kc < 9; ++kc)
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          z[i] = ((vm >> i) & 1ull) ? z[i] * a.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, z[i]);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16(tmem + b * 32, q_desc0 + static_cast<uint64_t>((kc * 8192 + ks * 32) >> 4),
+                      kb + static_cast<uint64_t>((kc * kKVChunk + ks * 32) >> 4), idesc_qk, (kc | ks) != 0);
+          tc_commit(&s_full[b]);
         }
-        float alpha = 1.0f;
-        if (m_run == -INFINITY) {
-          m_run = mt;                       // first tile with a valid key (O is still zero)
-        } else if (mt > m_run + 8.0f) {
-          alpha = exp2f(m_run - mt);
-          l_run *= alpha;
-          m_run = mt;
-          need_rescale = 1;
-        }
-        sAlpha[h] = alpha;
-        float lsum = 0.0f;
-        uint8_t* prow = sP + h * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = m_run == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * e] - m_run);
-            const float p1 = m_run == -INFINITY ? 0.0f : exp2f(z[8 * c + 2 * e + 1] - m_run);
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            const float2 pr = __bfloat1622float2(pb);   // the weights PV will use
-            lsum += pr.x + pr.y;
-            w[e] = *reinterpret_cast<const uint32_t*>(&pb);
-          }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        l_run += lsum;
-        fence_proxy_async_smem();
+        __syncwarp();
+        if (T >= 1 && !issue_pv(T - 1)) { good = false; break; }
       }
-    }
-    tc_fence_before();
-    const int any_rescale = __syncthreads_or(need_rescale);
-    ok = __syncthreads_and(got && ok);
-    if (!ok) break;
-
-    // ---- rare: rescale O^T columns by alpha[head]
-    if (any_rescale) {
-      tc_fence_after();
-      const uint32_t lane_base = tmem_O + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll 1
-      for (int d = 0; d < 4; ++d)
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          float v[32];
-          const uint32_t addr = lane_base + d * 64 + half * 32;
-          tmem_ld32(addr, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= sAlpha[half * 32 + i];
-          tmem_st32(addr, v);
+      if (good && !issue_pv(ntiles - 1)) good = false;
+      if (!good && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 10);
+        *abort_flag = 1;
+      }
+      if (elect_one()) {
+        tc_commit(drain);
+        wait_drain(drain, 0);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ producer
+      // Lane j owns row j of every tile. Its slot comes from the staged list; its five
+      // scales are loaded two tiles ahead into registers, so no global load sits on the
+      // per-tile path.
+      auto slot_of = [&](int T) {
+        const int i = T * kMlaTile + lane;
+        if (T >= ntiles) return -1;
+        if (list_in_smem) return static_cast<int>(sIdxList[i]);
+        int slot = i < nkeys ? phys[k0 + i] : -1;
+        if (slot < -1 || slot >= a.num_slots) {
+          record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(slot));
+          slot = -1;
         }
-      tc_fence_before();
-      __syncthreads();
-    }
-
-    // ---- PV
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t kv_base = smem_u32(sKV), p_base = smem_u32(sP);
+        return slot;
+      };
+      float sc_a[kKvGroups], sc_b[kKvGroups];   // scales of tiles T and T+1
+      auto load_scales = [&](int slot, float (&sc)[kKvGroups]) {
 #pragma unroll
-      for (int d = 0; d < 4; ++d)
+        for (int g = 0; g < kKvGroups; ++g)
+          sc[g] = (FP8 && slot >= 0) ? a.kv_scale[static_cast<int64_t>(slot) * kKvGroups + g] : 0.0f;
+      };
+      int slot_a = slot_of(0), slot_b = slot_of(1);
+      load_scales(slot_a, sc_a);
+      load_scales(slot_b, sc_b);
+      bool good = true;
+      for (int T = 0; T < ntiles; ++T) {
+        const int st = T % kMlaStages;
+        if (!wait_warp(&stage_empty[st], ((T / kMlaStages) & 1) ^ 1, abort_flag)) { good = false; break; }
+        uint8_t* meta = sStageMeta + st * kStageMetaBytes;
+        uint32_t* mult = reinterpret_cast<uint32_t*>(meta);            // [32][5]
+        int32_t* E = reinterpret_cast<int32_t*>(meta + 640);           // [32]
+        int32_t* slots = reinterpret_cast<int32_t*>(meta + 768);       // [32]
+        const int slot = slot_a;
+        if (FP8 && slot >= 0)
+          bulk_load(sStage + st * kStageRows + lane * kRowBytes, a.kv + static_cast<int64_t>(slot) * kRowBytes,
+                    kRowBytes, &stage_full[st]);
+        int Ej = 0;
+        if (FP8) {
+          float smax = 0.0f;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem_O + d * 64, sdesc_sw128(kv_base + (2 * d) * 8192 + ks * 2048, 8192, 1024),
-                  sdesc_sw128(p_base + ks * 32, 16, 1024), idesc_pv, (T > 0 || ks > 0) ? 1u : 0u);
-      tc_commit(o_done);
+          for (int g = 0; g < kKvGroups; ++g) smax = fmaxf(smax, sc_a[g]);
+          Ej = smax > 0.0f ? float_exponent(smax) : 0;
+          const float inv = exp2i(-Ej);
+#pragma unroll
+          for (int g = 0; g < kKvGroups; ++g) {
+            const __half2 m2 = __float2half2_rn(sc_a[g] * inv);
+            mult[lane * kKvGroups + g] = *reinterpret_cast<const uint32_t*>(&m2);
+          }
+        }
+        E[lane] = Ej;
+        slots[lane] = slot;
+        const unsigned vm = __ballot_sync(0xffffffffu, slot >= 0);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&stage_full[st], FP8 ? __popc(vm) * kRowBytes : 0u);
+        // rotate the two-tile lookahead
+        slot_a = slot_b;
+#pragma unroll
+        for (int g = 0; g < kKvGroups; ++g) sc_a[g] = sc_b[g];
+        slot_b = slot_of(T + 2);
+        load_scales(slot_b, sc_b);
+      }
+      if (!good && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 11);
+        *abort_flag = 1;
+      }
+      // bounded drain of this warp's outstanding row copies
+      if (lane == 0 && FP8)
+        for (int T = max(0, ntiles - kMlaStages); T < ntiles; ++T)
+          wait_drain(&stage_full[T % kMlaStages], (T / kMlaStages) & 1);
+      __syncwarp();
+    } else if (warp == 2 || warp == 3) {
+      // ------------------------------------------------------------ dequantisers
+      const int ct = tid - 64;   // 0..63
+      bool good = true;
+      for (int T = 0; T < ntiles; ++T) {
+        const int st = T % kMlaStages, b = T & 1;
+        if (!wait_warp(&stage_full[st], (T / kMlaStages) & 1, abort_flag)) { good = false; break; }
+        if (T >= 2 && !wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
+        const uint8_t* meta = sStageMeta + st * kStageMetaBytes;
+        const uint32_t* mult = reinterpret_cast<const uint32_t*>(meta);
+        const int32_t* slots = reinterpret_cast<const int32_t*>(meta + 768);
+        uint8_t* kv = sKV + b * kKVBytes;
+        if (FP8) {
+          const uint8_t* rows = sStage + st * kStageRows;
+#pragma unroll 3
+          for (int c = ct; c < kMlaTile * 36; c += 64) {
+            const int j = c / 36, cc = c - j * 36;
+            uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+            if (slots[j] >= 0) {
+              const uint4 raw = *reinterpret_cast<const uint4*>(rows + j * kRowBytes + cc * 16);
+              const uint32_t mw = mult[j * kKvGroups + (cc >> 3)];
+              const __half2 m2 = *reinterpret_cast<const __half2*>(&mw);
+              dequant4_f16(raw.x, m2, o0.x, o0.y);
+              dequant4_f16(raw.y, m2, o0.z, o0.w);
+              dequant4_f16(raw.z, m2, o1.x, o1.y);
+              dequant4_f16(raw.w, m2, o1.z, o1.w);
+            }
+            uint8_t* blk = kv + (cc >> 2) * kKVChunk;
+            *reinterpret_cast<uint4*>(blk + swz(j, (cc & 3) * 2)) = o0;
+            *reinterpret_cast<uint4*>(blk + swz(j, (cc & 3) * 2 + 1)) = o1;
+          }
+        } else {
+          for (int c = ct; c < kMlaTile * 72; c += 64) {
+            const int j = c / 72, cc = c - j * 72;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (slots[j] >= 0)
+              v = *reinterpret_cast<const uint4*>(a.kv + static_cast<int64_t>(slots[j]) * (2 * kDimK) + cc * 16);
+            *reinterpret_cast<uint4*>(kv + (cc >> 3) * kKVChunk + swz(j, cc & 7)) = v;
+          }
+        }
+        if (warp == 2) {   // row exponents and validity of this tile, for the softmax warps
+          const int32_t* E = reinterpret_cast<const int32_t*>(meta + 640);
+          int32_t* km = sKVMeta + b * 64;
+          km[lane] = E[lane];
+          const unsigned vm = __ballot_sync(0xffffffffu, slots[lane] >= 0);
+          if (lane == 0) km[32] = static_cast<int32_t>(vm);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&kv_full[b]);
+          mbar_arrive(&stage_empty[st]);
+        }
+      }
+      if (!good && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 12);
+        *abort_flag = 1;
+      }
+      __syncwarp();
+    } else {
+      // ------------------------------------------------------------ softmax group (warps 4..7)
+      const bool is_sm = warp < 6;            // warps 4,5: heads 0..63 = TMEM lanes 0..63
+      const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+      const int h = (warp - 4) * 32 + lane;   // head (meaningful for warps 4,5)
+      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+      float m_run = -INFINITY, l_run = 0.0f, cq = 0.0f;
+      int e_ref = kNoExp;                     // running max of the rows' exponents (same in every thread)
+      if (is_sm) cq = sCq[h];
+      bool good = true;
+      for (int T = 0; T < ntiles; ++T) {
+        const int b = T & 1;
+        float y[kMlaTile];
+        int need = 0;
+        if (is_sm) {
+          const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
+                           wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
+          if (got) {
+            tc_fence_after();
+            tmem_ld32(tmem + lane_base + b * 32, y);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[b]);
+            const int32_t* km = sKVMeta + b * 64;
+            const unsigned vm = static_cast<unsigned>(km[32]);
+            float ymax = -INFINITY;
+            int etile = kNoExp;
+#pragma unroll
+            for (int j = 0; j < kMlaTile; ++j) {
+              const bool v = (vm >> j) & 1u;
+              y[j] = v ? y[j] * cq * exp2i(km[j]) : -INFINITY;
+              ymax = fmaxf(ymax, y[j]);
+              if (v) etile = max(etile, km[j]);
+            }
+            float alpha = 1.0f;
+            if (vm != 0u) {
+              if (m_run == -INFINITY) {
+                m_run = ymax;                       // first tile with a valid row: nothing accumulated yet
+              } else if (ymax > m_run + 8.0f) {
+                alpha = exp2f(m_run - ymax);
+                l_run *= alpha;
+                m_run = ymax;
+              }
+              if (e_ref == kNoExp) {
+                e_ref = etile;
+              } else if (etile > e_ref) {
+                alpha *= exp2i(e_ref - etile);
+                e_ref = etile;
+              }
+            }
+            sAlpha[h] = alpha;
+            need = alpha != 1.0f ? 1 : 0;
+          } else {
+            good = false;
+          }
+        }
+        need = group_or(need);
+        good = group_and(good) != 0;
+        if (!good) break;
+        if (need) {
+          // rescale the O^T columns (heads) by alpha; PV(T-1) must have finished first
+          const bool got = wait_warp(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag);
+          if (got) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int d = 0; d < 4; ++d)
+#pragma unroll 1
+              for (int half = 0; half < 2; ++half) {
+                float v[32];
+                const uint32_t addr = tmem_O + lane_base + d * 64 + half * 32;
+                tmem_ld32(addr, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= sAlpha[half * 32 + i];
+                tmem_st32(addr, v);
+              }
+          }
+          good = group_and(got) != 0;
+          if (!good) break;
+        }
+        if (is_sm) {
+          // the P half this tile writes was last read by PV(T-2)
+          const bool got = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag);
+          if (got) {
+            const int32_t* km = sKVMeta + b * 64;
+            uint8_t* prow = sP + h * 128;
+            float lsum = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = 8 * c + 2 * e;
+                const float p0 = m_run == -INFINITY ? 0.0f : exp2f(y[j] - m_run);
+                const float p1 = m_run == -INFINITY ? 0.0f : exp2f(y[j + 1] - m_run);
+                lsum += p0 + p1;
+                if (FP8) {
+                  const float d0 = exp2i(km[j] - e_ref), d1 = exp2i(km[j + 1] - e_ref);
+                  __half2 hh = __floats2half2_rn(p0 * d0, p1 * d1);
+                  w[e] = *reinterpret_cast<uint32_t*>(&hh);
+                } else {
+                  __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+                  w[e] = *reinterpret_cast<uint32_t*>(&bb);
+                }
+              }
+              *reinterpret_cast<uint4*>(prow + (((b * 4 + c) ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            l_run += lsum;
+            fence_proxy_async_smem();
+          } else {
+            good = false;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        good = group_and(good) != 0;
+        if (!good) break;
+      }
+      // ---- epilogue: warps 4..7 read O^T (lanes = dims), softmax threads supply per-head scales
+      if (good) {
+        const bool split_out = a.nsplit > 1;
+        if (is_sm) {
+          const float l = l_run;
+          const float oscale = exp2i(e_ref == kNoExp ? 0 : e_ref);
+          sOutScale[h] = split_out ? oscale : (l > 0.0f ? oscale / l : 0.0f);
+          if (split_out) {
+            float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * 2;
+            ml[0] = l > 0.0f ? m_run : -INFINITY;
+            ml[1] = l;
+          } else if (a.lse != nullptr) {
+            a.lse[static_cast<int64_t>(q) * kHeads + h] =
+                l > 0.0f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          }
+        }
+        const int last = ntiles - 1;
+        const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag);
+        good = group_and(got) != 0;
+        if (good) {
+          tc_fence_after();
+          const int dim_in_tile = quarter * 32 + lane;
+#pragma unroll 1
+          for (int d = 0; d < 4; ++d) {
+            const int dim = d * 128 + dim_in_tile;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              tmem_ld32(tmem_O + lane_base + d * 64 + half * 32, v);
+#pragma unroll 4
+              for (int i = 0; i < 32; ++i) {
+                const int hh = half * 32 + i;
+                const float o = v[i] * sOutScale[hh];
+                if (split_out) {
+                  a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = o;
+                } else {
+                  const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
+                  if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
+                  else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
+                }
+              }
+            }
+          }
+        }
+      }
+      if (!good && lane == 0) {
+        record_error(a.err, DSA_ERR_TIMEOUT, 13);
+        *abort_flag = 1;
+      }
+      __syncwarp();
     }
-    got = wait_warp(o_done, T & 1, abort_flag);
-    tc_fence_after();
-    ok = __syncthreads_and(got && ok);
-    if (!ok) break;
   }
 
-  if (!ok) {
-    if (tid == 0) {
-      record_error(a.err, DSA_ERR_TIMEOUT, 4);
-      *abort_flag = 1;
-      // let this CTA's in-flight work land (bounded): its MMAs and its row copies
-      tc_commit(drain);
-      bounded_wait(drain, 0);
-      if (FP8)
-        for (int t = T; t < issued; ++t) bounded_wait(&stage_full[t & 1], (t >> 1) & 1);
-    }
-    __syncthreads();
-  } else {
-    // ---- epilogue
+  if (ntiles == 0) {
+    // nothing selected: zero output (or an empty partial)
     const bool split_out = a.nsplit > 1;
+    for (int i = tid; i < kHeads * kDimV; i += kMlaThreads) {
+      const int hh = i / kDimV, dim = i % kDimV;
+      if (split_out) {
+        a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = 0.0f;
+      } else {
+        const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
+        if (a.out_fp32) static_cast<float*>(a.out)[off] = 0.0f;
+        else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(0.0f);
+      }
+    }
     if (tid < kHeads) {
-      const float l = l_run;
-      sInvL[tid] = l > 0.0f ? 1.0f / l : 0.0f;
       if (split_out) {
         float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + tid) * 2;
-        ml[0] = l > 0.0f ? m_run : -INFINITY;
-        ml[1] = l;
+        ml[0] = -INFINITY;
+        ml[1] = 0.0f;
       } else if (a.lse != nullptr) {
-        a.lse[static_cast<int64_t>(q) * kHeads + tid] =
-            l > 0.0f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        a.lse[static_cast<int64_t>(q) * kHeads + tid] = -INFINITY;
       }
     }
-    __syncthreads();
-    const int dim_in_tile = warp * 32 + lane;
-#pragma unroll 1
-    for (int d = 0; d < 4; ++d) {
-      const int dim = d * 128 + dim_in_tile;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float v[32];
-        if (ntiles > 0) {
-          tmem_ld32(tmem_O + (static_cast<uint32_t>(warp * 32) << 16) + d * 64 + half * 32, v);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-        }
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const int h = half * 32 + i;
-          if (split_out) {
-            a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kDimV + dim] = v[i];
-          } else {
-            const float o = v[i] * sInvL[h];
-            const int64_t off = (static_cast<int64_t>(q) * kHeads + h) * kDimV + dim;
-            if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
-            else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
-          }
-        }
-      }
-    }
+  }
+  if (!ok && tid == 0) {
+    record_error(a.err, DSA_ERR_TIMEOUT, 14);
+    wait_drain(q_full, 0);   // the Q copy may still be landing
   }
 
   tc_fence_before();
@@ -444,5 +670,7 @@ cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cu
   ++*launches;
   return cudaGetLastError();
 }
+
+int mla_tile_keys() { return kMlaTile; }
 
 }  // namespace dsa

@@ -99,7 +99,7 @@ typedef struct {
  *  scores   device [B*n_q, L_max] fp32 output; entries s < vis(q) are written, the rest
  *           are left untouched. L_max >= max_pages_per_seq*64 is not required, but
  *           vis(q) is clamped to L_max.
- *  Alignment: q_idx, k_cache 16-byte aligned; L_max >= 1.
+ *  Alignment: q_idx, k_cache and k_scale 16-byte aligned; L_max >= 1.
  */
 dsa_status dsa_indexer_scores(const dsa_paging* paging,
                               const void* q_idx, dsa_dtype q_dtype, const float* q_scale,

@@ -43,13 +43,13 @@ DV = 512
 # ----------------------------------------------------------------------------------
 # storage formats
 
-def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+def _e4m3_value(c: np.ndarray) -> np.ndarray:
     """OCP FP8 E4M3 ("fn" variant) code -> exact fp64 value.
 
     1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits. Exponent field 0 is
     subnormal (value = m/8 * 2^-6). There is no infinity; S.1111.111 is NaN, so the
     largest finite magnitude is 1.75 * 2^8 = 448."""
-    c = np.asarray(codes).astype(np.int64)
+    c = np.asarray(c).astype(np.int64)
     sign = np.where((c >> 7) & 1, -1.0, 1.0)
     e = (c >> 3) & 0xF
     m = (c & 0x7).astype(np.float64)
@@ -57,6 +57,14 @@ def decode_e4m3(codes: np.ndarray) -> np.ndarray:
     sub = np.ldexp(m / 8.0, -6)
     v = sign * np.where(e == 0, sub, normal)
     return np.where((e == 0xF) & ((c & 0x7) == 0x7), np.nan, v)
+
+
+_E4M3 = _e4m3_value(np.arange(256))   # the definition evaluated once for every code
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes -> exact fp64 values (lookup in the 256-entry table of _e4m3_value)."""
+    return _E4M3[np.asarray(codes, dtype=np.uint8)]
 
 
 def decode_bf16(bits: np.ndarray) -> np.ndarray:
@@ -146,14 +154,15 @@ def indexer_scores(case: dict, queries=None) -> np.ndarray:
     Q = dequant_index_queries(case)
     w = case["head_w"].astype(np.float64)
     out = np.full((len(queries), L_max), -np.inf)
+    chunk = 65536                                            # tokens per step (memory only)
     for i, q in enumerate(queries):
         v = int(vis[q])
-        if v == 0:
-            continue
-        slots = physical_slots(case["block_table"][q // case["n_q"]], np.arange(v))
-        K = dequant_index_keys(case, slots)                 # [v, 128]
-        logits = Q[q] @ K.T                                  # [64, v]
-        out[i, :v] = (w[q][:, None] * np.maximum(logits, 0.0)).sum(axis=0)
+        for s0 in range(0, v, chunk):
+            s1 = min(v, s0 + chunk)
+            slots = physical_slots(case["block_table"][q // case["n_q"]], np.arange(s0, s1))
+            K = dequant_index_keys(case, slots)             # [n, 128]
+            logits = Q[q] @ K.T                              # [64, n]
+            out[i, s0:s1] = (w[q][:, None] * np.maximum(logits, 0.0)).sum(axis=0)
     return out
 
 

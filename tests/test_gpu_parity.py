@@ -126,3 +126,47 @@ def test_split_count_independence():
     one, _, _ = g.mla(phys[:1])              # 1 query  -> even more splits
     assert dsa.mla_num_splits(1, case["top_k"]) != dsa.mla_num_splits(8, case["top_k"])
     assert np.max(np.abs(full[0] - one[0])) <= 2e-3
+
+
+def _topk_on_scores(scores_np, vis, top_k, seed=40):
+    """Runs dsa_topk_pagemap on caller-chosen fp32 scores (one query per row)."""
+    import torch
+    import deepseek_sparse_attention_head_b200 as dsa
+    from tests.gpu_path import GpuCase
+    B, L = scores_np.shape
+    case = generate(CaseSpec("topk_custom", tuple(int(v) for v in vis), top_k=top_k, n_planted=0, seed=seed,
+                             max_pages=(L + 63) // 64))
+    g = GpuCase(case)
+    s = torch.from_numpy(np.ascontiguousarray(scores_np.astype(np.float32))).cuda()
+    lo, ph, err = g.topk(s, top_k)
+    return case, lo, ph, err
+
+
+def test_topk_ties_and_candidate_overflow():
+    """Constant and few-valued rows put every key in one first-digit bin, overflowing the
+    shared-memory candidate buffer and taking the global-refinement path."""
+    rng = np.random.default_rng(3)
+    L = 20032
+    rows = [np.full(L, 0.5), rng.choice([0.25, 0.5, 1.0], size=L), rng.standard_normal(L) * 1e-3 + 7.0,
+            np.linspace(-3, 3, L)[rng.permutation(L)], -np.abs(rng.standard_normal(L))]
+    scores = np.stack(rows)
+    vis = np.array([L, L - 5, 19000, L, 12345])
+    case, lo, ph, err = _topk_on_scores(scores, vis, 777)
+    assert err == 0
+    for i in range(len(rows)):
+        check_topk_exact(lo[i], scores[i].astype(np.float32), vis[i], 777)
+    assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
+
+
+def test_topk_extreme_values():
+    rng = np.random.default_rng(4)
+    L = 4096
+    base = rng.standard_normal((3, L)).astype(np.float32)
+    base[0, ::7] = np.float32(3.0e38)
+    base[1, ::5] = -np.float32(3.0e38)
+    base[2, :] = np.float32(1e-40) * rng.integers(-5, 5, L)   # subnormals and zeros of both signs
+    vis = np.array([L, L, 4000])
+    case, lo, ph, err = _topk_on_scores(base, vis, 300)
+    assert err == 0
+    for i in range(3):
+        check_topk_exact(lo[i], base[i], vis[i], 300)
