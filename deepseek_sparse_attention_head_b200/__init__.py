@@ -73,7 +73,7 @@ _SIGNATURES = {
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is missing: build it with "
-                          "`python -m deepseek_sparse_attention_head_b200.build` (needs nvcc)")
+                          "`python deepseek_sparse_attention_head_b200/build.py` (needs nvcc)")
     lib = ctypes.CDLL(_LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
         fn = getattr(lib, name)

@@ -1,6 +1,6 @@
 """Builds libdsa_b200.so in-tree for sm_100a (nvcc; no torch extension machinery).
 
-    python -m deepseek_sparse_attention_head_b200.build [--verbose]
+    python deepseek_sparse_attention_head_b200/build.py [--verbose] [--ptxas]
 """
 from __future__ import annotations
 
