@@ -59,6 +59,8 @@ _SIGNATURES = {
     "dsa_topk_pagemap": (_i32, [_PP, _vp, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
     "dsa_pagemap": (_i32, [_PP, _vp, _i32, _vp, _vp, _sz, _vp]),
     "mla_sparse_decode": (_i32, [_i32, _vp, _vp, _i32, _vp, _i64, _vp, _i32, _f32, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "mla_sparse_decode_noalloc": (_i32, [_i32, _vp, _vp, _i32, _vp, _i64, _vp, _i32, _f32, _vp, _i32, _vp, _vp,
+                                         _vp]),
     "dsa_decode_layer": (_i32, [_PP, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _i32,
                                 _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_workspace_size": (_sz, [_PP, _i64, _i32, _i32]),
@@ -219,6 +221,21 @@ def mla_sparse_decode(q: torch.Tensor, kv_cache: torch.Tensor, kv_scale, physica
                                 float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(lse), _ptr(workspace),
                                 workspace.numel(), _stream(stream))
     _check(st, "mla_sparse_decode")
+    return out
+
+
+def mla_sparse_decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, kv_scale, physical: torch.Tensor,
+                              softmax_scale: float, out: torch.Tensor, lse=None, status=None, stream=None):
+    """mla_sparse_decode with its scratch in the library's own device array (no workspace).
+
+    For callers that cannot allocate device memory. `status`, if given, is a device int32
+    tensor of 2 elements that receives the call's device-side error words."""
+    Bq = int(q.shape[0])
+    st = _lib.mla_sparse_decode_noalloc(Bq, _ptr(q), _ptr(kv_cache), _dtype_code(kv_cache), _ptr(kv_scale),
+                                        int(kv_cache.shape[0]), _ptr(physical), int(physical.shape[-1]),
+                                        float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(lse),
+                                        _ptr(status), _stream(stream))
+    _check(st, "mla_sparse_decode_noalloc")
     return out
 
 

@@ -399,3 +399,68 @@ const char* dsa_status_string(dsa_status status) {
 int32_t dsa_last_launch_count(void) { return g_launches; }
 
 }  // extern "C"
+
+// ====================================================================== MLA decode without allocation
+//
+// mla_sparse_decode_noalloc: the split-KV MLA decode with its partials (and error words)
+// kept in one file-scope device array instead of a caller-provided workspace, for callers
+// that cannot allocate device memory themselves (a plugin inside an engine that owns the
+// GPU's memory, or a loop that must not pay for cudaMalloc).
+
+namespace {
+
+// Largest layout mla_sparse_decode ever needs on a 148-SM GPU: 148 (query, split) pairs of
+// 64 x 512 fp32 partial outputs plus 64 x 2 (max, sum) floats, and the 256-byte header.
+constexpr size_t kMlaStaticScratchBytes = size_t(20) << 20;
+
+}  // namespace
+
+// One copy per device that loads this library, held until the process exits.
+static __device__ __align__(256) uint8_t g_mla_static_scratch[kMlaStaticScratchBytes];
+
+namespace {
+
+// Device address of g_mla_static_scratch on the current device. In host code the array's
+// name is only a handle, so the address is looked up once per device, with that device
+// current, on the first call made there.
+uint8_t* mla_static_scratch() {
+  static std::mutex mu;
+  static uint8_t* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_mla_static_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" dsa_status mla_sparse_decode_noalloc(int32_t Bq, const void* q, const void* kv_cache,
+                                                dsa_dtype kv_dtype, const float* kv_scale, int64_t num_slots,
+                                                const int32_t* physical, int32_t top_k, float softmax_scale,
+                                                void* out, dsa_dtype out_dtype, float* lse, unsigned int* status,
+                                                void* stream) {
+  g_launches = 0;
+  dsa_status s = check_mla_inputs(Bq, q, kv_cache, kv_dtype, kv_scale, num_slots, physical, top_k, softmax_scale,
+                                  out, out_dtype);
+  if (s != DSA_OK) return s;
+  if (status != nullptr && !aligned(status, 8)) return DSA_ERR_INVALID_ARG;
+  int kps = 0;
+  const int nsplit = mla_splits_for(Bq, top_k, &kps);
+  const Layout lay = layout_for(0, Bq, 0, top_k, -1, nsplit);
+  if (lay.total > kMlaStaticScratchBytes) return DSA_ERR_WORKSPACE;
+  uint8_t* scratch = mla_static_scratch();
+  if (scratch == nullptr) return DSA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The error words must read zero when the kernels start; the partials are always
+  // written in full before the combine reads them.
+  if (cudaMemsetAsync(scratch, 0, 8, st) != cudaSuccess) return DSA_ERR_CUDA;
+  s = run_mla(Bq, q, kv_cache, kv_dtype, kv_scale, num_slots, physical, top_k, softmax_scale, out, out_dtype, lse,
+              scratch, lay, nsplit, kps, st);
+  if (s != DSA_OK || status == nullptr) return s;
+  return cuda_status(cudaMemcpyAsync(status, scratch, 8, cudaMemcpyDeviceToDevice, st));
+}

@@ -153,6 +153,32 @@ dsa_status mla_sparse_decode(int32_t Bq, const void* q, const void* kv_cache, ds
                              void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * mla_sparse_decode without a workspace argument, for callers that cannot allocate
+ * device memory themselves: a plugin running inside an engine that reserves and owns all
+ * of the GPU's memory and hands out none of it, or a decode loop that must not call
+ * cudaMalloc and cudaFree, which can synchronise the whole device. The paper has no counterpart to this entry point; it is a packaging of
+ * stage 3 only. Arguments and results are those of mla_sparse_decode, except:
+ *  status  optional device [2] uint32 (8-byte aligned), or NULL: receives this call's
+ *          device-side error words; read and clear it with dsa_get_error(status, stream).
+ *          With NULL, device-side range and timeout errors are not reported.
+ * The split partials live in a 20 MiB array that the library defines in device memory;
+ * every GPU that loads the library holds it until the process exits. That covers every
+ * (Bq, top_k) on a 148-SM B200; a call whose partials would not fit (a GPU with more SMs)
+ * returns DSA_ERR_WORKSPACE. The first call on each device looks up the array's device
+ * address (with that device current), so make that call before any stream capture.
+ * All calls on a device share the array and it keeps the last call's contents: calls that
+ * may overlap on the GPU (different streams, no ordering between them) race and corrupt
+ * each other's results. Allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine); each call enqueues one 8-byte memset, the kernels of mla_sparse_decode and,
+ * with a status pointer, one 8-byte device-to-device copy.
+ */
+dsa_status mla_sparse_decode_noalloc(int32_t Bq, const void* q, const void* kv_cache, dsa_dtype kv_dtype,
+                                     const float* kv_scale, int64_t num_slots,
+                                     const int32_t* physical, int32_t top_k, float softmax_scale,
+                                     void* out, dsa_dtype out_dtype, float* lse,
+                                     unsigned int* status, void* stream);
+
+/*
  * The fused decode layer: indexer -> top-k + page map -> MLA sparse decode on one
  * stream, intermediate scores and index lists kept in the workspace. Arguments as
  * in the three stages above (q_idx and k_cache share idx_dtype). The scores row

@@ -109,3 +109,14 @@ def test_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError):
         dsa._ptr(torch.zeros(4))
+
+
+def test_noalloc_argument_errors():
+    def call(Bq=2, top_k=64, q=FAKE, scale=0.07, status=None):
+        return _lib.mla_sparse_decode_noalloc(Bq, q, FAKE, dsa.DSA_FP8_E4M3, FAKE, 1024, FAKE, top_k, scale, FAKE,
+                                              dsa.DSA_BF16, None, status, None)
+    assert call(Bq=0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(q=None) == dsa.DSA_ERR_INVALID_ARG
+    assert call(top_k=16385) == dsa.DSA_ERR_INVALID_ARG
+    assert call(scale=0.0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(status=ctypes.c_void_p(0x100004)) == dsa.DSA_ERR_INVALID_ARG   # status words need 8-byte alignment
