@@ -5,20 +5,23 @@
 //
 // (576 = 512 latent + 64 rope columns; "Show HN: colibri", features.)
 //
-// Design (sm_100a): grid = (query, split); a CTA walks 32-row tiles of its share of
-// the index list with warp-specialised, double-buffered stages:
-//   warp 1    producer: the tile's slot ids, one 576-byte bulk async copy per fp8 row
-//             into a 3-deep ring, and the row's five scales folded into an exact
-//             power-of-two row exponent E_j plus five fp16 multipliers s_g / 2^E_j;
-//   warps 2-3 dequantisers: fp8 code -> fp16 (exact) x multiplier -> fp16 tile,
-//             128-byte swizzled; the tile is the K operand of QK (K-major) and the
-//             V operand of PV (MN-major) at once;
-//   warp 0    tcgen05 issuer:  S = Q' K'^T (M=128, rows 64..127 unused, N=32),
-//             O^T += V'^T P'^T (4 x M=128, N=64); fp32 accumulators in TMEM;
-//   warps 4-5 softmax, one thread per head (its TMEM lane): running max with lazy
-//             rescaling (only when a tile's max exceeds it by more than 8 in log2
-//             units), exact fp32 normaliser, fp16 weights P' = p * 2^(E_j - E_ref);
-//   warps 4-7 the rare O rescale and the output epilogue (all 128 TMEM lanes).
+// Design (sm_100a): grid = (query, split); a CTA walks 64-row tiles of its share of the
+// index list through two tile buffers, with warp-specialised roles:
+//   warps 5-10 loaders, two groups of three: group g fills buffer g with tiles g, g+2, ...
+//             Each thread keeps 24 sixteen-byte pieces of its group's next tile in flight
+//             (plain global loads issued a tile pair ahead), then turns fp8 codes into
+//             fp16 (exact) x a per-row multiplier s_g / 2^E_j and stores them 128-byte
+//             swizzled: the tile is the K operand of QK (K-major) and the V operand of PV
+//             (MN-major) at once. E_j is the row's power-of-two exponent.
+//   warp 4    tcgen05 issuer: S = Q' K'^T (M=128, rows 64..127 unused, N=64 keys),
+//             O^T += V'^T P'^T (4 x M=128 dims, N=64 heads); fp32 accumulators in TMEM.
+//             Issue order QK(t), QK(t+1), PV(t), PV(t+1) lets one buffer refill while the
+//             other tile's MMAs run.
+//   warps 0-1 softmax, one thread per head (its TMEM lane): running max with lazy
+//             rescaling (only when a tile's max exceeds it by more than 8 in log2 units),
+//             exact fp32 normaliser, fp16 weights P' = p * 2^(E_j - E_ref) written into
+//             the tile's rope chunk, which QK has finished with.
+//   warps 0-3 Q rescale at the start, the rare O rescale and the output epilogue.
 // Q is staged once per CTA and rescaled per head by a power of two into fp16. With
 // a bf16 cache the same pipeline runs in bf16 without any rescaling.
 // Splits write (m, l, o) partials that mla_combine_kernel merges by log-sum-exp.
@@ -30,52 +33,57 @@
 
 namespace dsa {
 
-constexpr int kMlaTile = 32;
-constexpr int kMlaThreads = 256;
-constexpr int kMlaStages = 3;
-constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,64); O^T: cols [64, 320)
-constexpr int kRowBytes = kDimK;              // fp8 row
-constexpr int kStageRows = kMlaTile * kRowBytes;
+constexpr int kMlaTile = 64;
+constexpr int kMlaWarps = 11;
+constexpr int kMlaThreads = kMlaWarps * 32;
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp0 = 5;                 // loader group g: warps 5 + 3g .. 7 + 3g
+constexpr int kLoadThreads = 96;              // per group
+constexpr int kBatchPieces = 24;              // 16-byte pieces per loader thread and batch
+constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,128); O^T: cols [128, 384)
+constexpr uint32_t kTmemO = 128;
 constexpr int kNoExp = -100000;               // "no valid row seen yet"
+constexpr int kKVChunk = kMlaTile * 128;      // one 64-column chunk of a tile
+constexpr int kKVBytes = 9 * kKVChunk;
+constexpr int kPChunk = 8;                    // the rope chunk, reused for P after QK
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr int kOffQ = 0;                                        // 9 x [64 x 128 B]
-constexpr int kOffStage = kOffQ + 9 * 8192;                     // 3 x [32 x 576 B]
-constexpr int kOffStageMeta = kOffStage + kMlaStages * kStageRows;
-constexpr int kStageMetaBytes = 1024;                           // mult[32][5] u32, E[32], slot[32]
-constexpr int kOffKV = kOffStageMeta + kMlaStages * kStageMetaBytes;   // 2 x 9 x [32 x 128 B]
-constexpr int kKVChunk = kMlaTile * 128;
-constexpr int kKVBytes = 9 * kKVChunk;
-constexpr int kOffP = kOffKV + 2 * kKVBytes;                    // [64 heads x 128 B]; tile parity picks the half
-constexpr int kOffKVMeta = kOffP + 8192;                        // 2 x (E[32], vmask)
-constexpr int kOffHead = kOffKVMeta + 512;                      // cq[64], alpha[64], outscale[64]
-constexpr int kOffIdxList = kOffHead + 768;                     // the split's slot list (<= 2048 entries)
-constexpr int kIdxListCap = 2048;
-constexpr int kOffBars = kOffIdxList + kIdxListCap * 4;
+constexpr int kOffKV = kOffQ + 9 * 8192;                        // 2 x 9 x [64 x 128 B]
+constexpr int kOffKVMeta = kOffKV + 2 * kKVBytes;               // 2 x per-key tables (KVMeta)
+constexpr int kKVMetaBytes = 1152;
+constexpr int kOffGrpMeta = kOffKVMeta + 2 * kKVMetaBytes;      // 2 x mult[64][5] (fp16x2)
+constexpr int kGrpMetaBytes = kMlaTile * kKvGroups * 4;
+constexpr int kOffHead = kOffGrpMeta + 2 * kGrpMetaBytes;       // cq[64], alpha[64], outscale[64]
+constexpr int kOffBars = kOffHead + 768;
 constexpr int kOffMisc = kOffBars + 256;
-constexpr int kMlaSmem = kOffMisc + 64 + 1024;
+constexpr int kOffIdxList = kOffMisc + 64;                      // the split's slot list
+constexpr int kIdxListCap = 1024;
+constexpr int kMlaSmem = kOffIdxList + kIdxListCap * 4 + 1024;
 
-static_assert(kOffKV % 1024 == 0 && kOffP % 1024 == 0 && kOffStage % 16 == 0, "alignment");
+static_assert(kOffKV % 1024 == 0 && kKVBytes % 1024 == 0, "alignment");
+static_assert(kIdxListCap % kMlaTile == 0, "list capacity");
 static_assert(kMlaSmem <= 232448, "shared memory");
+static_assert(kLoadThreads * kBatchPieces == kMlaTile * 36, "an fp8 tile is one batch");
 
-// OR / AND over the 128 threads of warps 4..7 (named barrier 1).
-__device__ __forceinline__ int group_or(int v) {
+// bar.red over named barrier `id` of `count` threads: OR / AND of a predicate.
+__device__ __forceinline__ int bar_or(int id, int count, int v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.or.pred q, %1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
       : "memory");
   return static_cast<int>(r);
 }
-__device__ __forceinline__ int group_and(int v) {
+__device__ __forceinline__ int bar_and(int id, int count, int v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.and.pred q, %1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}\n"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v))
+      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
       : "memory");
   return static_cast<int>(r);
 }
@@ -91,6 +99,27 @@ __device__ __forceinline__ int float_exponent(float s) {  // floor(log2 s) for p
 __device__ __forceinline__ float exp2i(int e) {  // exact 2^e, clamped to the normal fp32 range
   e = e < -126 ? -126 : (e > 127 ? 127 : e);
   return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+// Per-key tables of one tile buffer, written by the loaders (row j of the tile):
+//   kmul[j] = 2^E_j (0 for an unused row), kadd[j] = 0 (-inf for an unused row),
+//   E[j] = the row exponent, emax[w] = max E over the valid rows j in [32w, 32w+32)
+//   (kNoExp when none), vmask[w] = validity bits of those rows;
+// and by the softmax threads: fac[j] = 2^(E_j - E_ref) (0 for an unused row).
+struct KVMeta {
+  float kmul[64];
+  float kadd[64];
+  int32_t E[64];
+  float fac[64];
+  uint32_t vmask[2];
+  int32_t emax[2];
+};
+static_assert(sizeof(KVMeta) <= 1152, "tile table size");
+
+__device__ __forceinline__ float ex2_ftz(float x) {  // hardware 2^x; tiny results flush to zero
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Four E4M3 codes -> four fp16 (exact) times the fp16 multiplier pair m2.
@@ -109,25 +138,22 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sStage = smem + kOffStage;
-  uint8_t* sStageMeta = smem + kOffStageMeta;
   uint8_t* sKV = smem + kOffKV;
-  uint8_t* sP = smem + kOffP;
-  int32_t* sKVMeta = reinterpret_cast<int32_t*>(smem + kOffKVMeta);
+  KVMeta* sKVMeta = reinterpret_cast<KVMeta*>(smem + kOffKVMeta);
+  uint32_t* sGrpMeta = reinterpret_cast<uint32_t*>(smem + kOffGrpMeta);
   float* sCq = reinterpret_cast<float*>(smem + kOffHead);
   float* sAlpha = sCq + 64;
   float* sOutScale = sCq + 128;
   int32_t* sIdxList = reinterpret_cast<int32_t*>(smem + kOffIdxList);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* stage_full = bars + 1;    // [3]
-  uint64_t* stage_empty = bars + 4;   // [3]
-  uint64_t* kv_full = bars + 7;       // [2]
-  uint64_t* s_full = bars + 9;        // [2]
-  uint64_t* s_empty = bars + 11;      // [2]
-  uint64_t* p_full = bars + 13;       // [2]
-  uint64_t* pv_done = bars + 15;      // [2]
-  uint64_t* drain = bars + 17;
+  uint64_t* q_ready = bars + 1;
+  uint64_t* kv_full = bars + 2;       // [2]
+  uint64_t* s_full = bars + 4;        // [2]
+  uint64_t* s_empty = bars + 6;       // [2]
+  uint64_t* p_full = bars + 8;        // [2]
+  uint64_t* pv_done = bars + 10;      // [2]
+  uint64_t* drain = bars + 12;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -144,12 +170,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < kMlaStages; ++i) {
-      mbar_init(&stage_full[i], 1);
-      mbar_init(&stage_empty[i], 2);
-    }
+    mbar_init(q_ready, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 2);
+      mbar_init(&kv_full[i], 3);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 2);
       mbar_init(&p_full[i], 4);
@@ -159,7 +182,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, kMlaTmemCols);
     tmem_relinquish();
   }
@@ -167,10 +190,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_O = tmem + 64;
 
-  // the split's slot list, staged once (invalid entries become -1)
-  const bool list_in_smem = nkeys <= kIdxListCap;
+  if (ntiles > 0 && tid == 0) {
+    tma_prefetch_map(&tmap_q);
+    mbar_arrive_expect_tx(q_full, 9u * 8192u);
+    for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
+  }
+
+  // the split's slot list, staged once when it fits (invalid entries become -1)
+  const bool list_in_smem = ntiles * kMlaTile <= kIdxListCap;
   if (list_in_smem) {
     for (int i = tid; i < ntiles * kMlaTile; i += kMlaThreads) {
       int slot = i < nkeys ? phys[k0 + i] : -1;
@@ -181,411 +209,413 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       sIdxList[i] = slot;
     }
   }
-
-  // ---------------------------------------------------------------- Q: load, rescale per head
-  bool ok = true;
-  if (ntiles > 0) {
-    if (tid == 0) {
-      tma_prefetch_map(&tmap_q);
-      mbar_arrive_expect_tx(q_full, 9u * 8192u);
-      for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
+  __syncthreads();
+  auto slot_at = [&](int T, int row) -> int {
+    const int i = T * kMlaTile + row;
+    if (list_in_smem) return sIdxList[i];
+    int slot = i < nkeys ? phys[k0 + i] : -1;
+    if (slot < -1 || slot >= a.num_slots) {
+      record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(slot));
+      slot = -1;
     }
-    ok = wait_warp(q_full, 0, abort_flag);
-    const int h = tid >> 2, part = tid & 3;   // 4 threads per head, 18 of its 72 16-byte units each
-    int F = 0;
-    if (FP8 && ok) {
-      float mx = 0.0f;
-      for (int u = part * 18; u < part * 18 + 18; ++u) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      F = mx > 0.0f ? float_exponent(mx) : 0;
-      const float inv = exp2i(-F);
-      for (int u = part * 18; u < part * 18 + 18; ++u) {
-        uint4* p = reinterpret_cast<uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
-        const uint4 v = *p;
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-          __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
-          w[i] = *reinterpret_cast<uint32_t*>(&hh);
-        }
-        *p = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-    if (part == 0) sCq[h] = a.scale_log2 * exp2i(F);
-    fence_proxy_async_smem();
-  }
-  ok = __syncthreads_and(ok) != 0;
+    return slot;
+  };
 
   // fp16 operands for an fp8 cache, bf16 for a bf16 cache
   const uint32_t fmt = FP8 ? 0u : 1u;
-  const uint32_t idesc_qk = idesc_make(fmt, fmt, false, false, 128, kMlaTile);
-  const uint32_t idesc_pv = idesc_make(fmt, fmt, true, false, 128, 64);
 
-  if (ok && ntiles > 0) {
-    if (warp == 0) {
-      // ------------------------------------------------------------ tcgen05 issuer (whole warp)
-      // Descriptors are formed once and advanced by constants; MMAs and commits come from
-      // one elected lane of the converged warp.
-      bool good = true;
-      const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);                 // K-major view
-      const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);            // MN-major view
-      const uint64_t p_desc0 = sdesc_sw128(smem_u32(sP), 16, 1024);
-      auto issue_pv = [&](int T) {
-        const int b = T & 1;
-        if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint64_t vb = v_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
-        const uint64_t pb = p_desc0 + static_cast<uint64_t>((b * 64) >> 4);
-        if (elect_one()) {
+  if (ntiles > 0 && warp < 4) {
+    // ---------------------------------------------------------------- Q rescale, softmax, epilogue
+    bool good = wait_warp(q_full, 0, abort_flag);
+    const bool q_landed = good;
+    {
+      const int h = tid >> 1, part = tid & 1;   // 2 threads per head, 36 of its 72 16-byte units each
+      int F = 0;
+      if (FP8 && good) {
+        float mx = 0.0f;
+        for (int u = part * 36; u < part * 36 + 36; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        F = mx > 0.0f ? float_exponent(mx) : 0;
+        const float inv = exp2i(-F);
+        for (int u = part * 36; u < part * 36 + 36; ++u) {
+          uint4* p = reinterpret_cast<uint4*>(sQ + (u >> 3) * 8192 + swz(h, u & 7));
+          const uint4 v = *p;
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
+            w[i] = *reinterpret_cast<uint32_t*>(&hh);
+          }
+          *p = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      if (part == 0) sCq[h] = a.scale_log2 * exp2i(F);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    good = bar_and(1, 128, good) != 0;
+
+    const bool is_sm = warp < 2;            // warps 0,1: heads 0..63 = TMEM lanes 0..63
+    const int h = warp * 32 + lane;         // head (meaningful for warps 0,1)
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.0f, cq = 0.0f;
+    int e_ref = kNoExp;                     // running max of the rows' exponents (same in every thread)
+    if (is_sm) cq = sCq[h];
+    for (int T = 0; T < ntiles && good; ++T) {
+      const int b = T & 1;
+      KVMeta* km = sKVMeta + b;
+      float y[kMlaTile];
+      int need = 0;
+      if (is_sm) {
+        const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
+                         wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
+        if (got) {
+          tc_fence_after();
+          tmem_ld64(tmem + lane_base + b * kMlaTile, y);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_empty[b]);
+          // logits in log2 units: z = acc * cq * 2^E_j, -inf for unused rows
+          float ymax = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < kMlaTile; j += 4) {
+            const float4 mu = *reinterpret_cast<const float4*>(&km->kmul[j]);
+            const float4 ad = *reinterpret_cast<const float4*>(&km->kadd[j]);
+            y[j + 0] = fmaf(y[j + 0], cq * mu.x, ad.x);
+            y[j + 1] = fmaf(y[j + 1], cq * mu.y, ad.y);
+            y[j + 2] = fmaf(y[j + 2], cq * mu.z, ad.z);
+            y[j + 3] = fmaf(y[j + 3], cq * mu.w, ad.w);
+            ymax = fmaxf(fmaxf(ymax, fmaxf(y[j + 0], y[j + 1])), fmaxf(y[j + 2], y[j + 3]));
+          }
+          const int etile = max(km->emax[0], km->emax[1]);
+          float alpha = 1.0f;
+          if ((km->vmask[0] | km->vmask[1]) != 0u) {
+            if (m_run == -INFINITY) {
+              m_run = ymax;                       // first tile with a valid row: nothing accumulated yet
+            } else if (ymax > m_run + 8.0f) {
+              alpha = exp2f(m_run - ymax);
+              l_run *= alpha;
+              m_run = ymax;
+            }
+            if (e_ref == kNoExp) {
+              e_ref = etile;
+            } else if (etile > e_ref) {
+              alpha *= exp2i(e_ref - etile);
+              e_ref = etile;
+            }
+          }
+          // this thread also owns key h of the tile: its P' factor 2^(E_h - E_ref)
+          km->fac[h] = km->kadd[h] == 0.0f ? exp2i(km->E[h] - e_ref) : 0.0f;
+          sAlpha[h] = alpha;
+          need = alpha != 1.0f ? 1 : 0;
+        } else {
+          good = false;
+        }
+      }
+      need = bar_or(1, 128, need);
+      good = bar_and(1, 128, good) != 0;
+      if (!good) break;
+      if (need) {
+        // rescale the O^T columns (heads) by alpha; PV(T-1) must have finished first
+        const bool got = wait_warp(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag);
+        if (got) {
+          tc_fence_after();
+#pragma unroll 1
           for (int d = 0; d < 4; ++d)
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              const uint32_t addr = tmem + kTmemO + lane_base + d * 64 + half * 32;
+              tmem_ld32(addr, v);
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-              mma_f16(tmem_O + d * 64, vb + static_cast<uint64_t>(((2 * d) * kKVChunk + ks * 2048) >> 4),
-                      pb + static_cast<uint64_t>((ks * 32) >> 4), idesc_pv, (T > 0 || ks > 0) ? 1u : 0u);
-          tc_commit(&pv_done[b]);
+              for (int i = 0; i < 32; ++i) v[i] *= sAlpha[half * 32 + i];
+              tmem_st32(addr, v);
+            }
         }
-        __syncwarp();
-        return true;
-      };
-      for (int T = 0; T < ntiles; ++T) {
-        const int b = T & 1;
-        if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag)) { good = false; break; }
-        if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
+        good = bar_and(1, 128, got) != 0;
+        if (!good) break;
+      }
+      if (is_sm) {
+        // p = 2^(z - m) (fp32, summed exactly into l); P' = p * 2^(E_j - E_ref) in the
+        // tile's rope chunk (K-major rows of 64 keys per head)
+        uint8_t* prow = sKV + b * kKVBytes + kPChunk * kKVChunk + h * 128;
+        const float mm = m_run == -INFINITY ? 0.0f : m_run;
+        float lsum0 = 0.0f, lsum1 = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 f0 = *reinterpret_cast<const float4*>(&km->fac[8 * c]);
+          const float4 f1 = *reinterpret_cast<const float4*>(&km->fac[8 * c + 4]);
+          const float fa[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 8 * c + 2 * e;
+            const float p0 = ex2_ftz(y[j] - mm);
+            const float p1 = ex2_ftz(y[j + 1] - mm);
+            lsum0 += p0;
+            lsum1 += p1;
+            if (FP8) {
+              __half2 hh = __floats2half2_rn(p0 * fa[2 * e], p1 * fa[2 * e + 1]);
+              w[e] = *reinterpret_cast<uint32_t*>(&hh);
+            } else {
+              __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+              w[e] = *reinterpret_cast<uint32_t*>(&bb);
+            }
+          }
+          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l_run += lsum0 + lsum1;
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[b]);
+    }
+    // ---- epilogue: warps 0..3 read O^T (lanes = dims), softmax threads supply per-head scales
+    if (good) {
+      const bool split_out = a.nsplit > 1;
+      if (is_sm) {
+        const float l = l_run;
+        const float oscale = exp2i(e_ref == kNoExp ? 0 : e_ref);
+        sOutScale[h] = split_out ? oscale : (l > 0.0f ? oscale / l : 0.0f);
+        if (split_out) {
+          float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * 2;
+          ml[0] = l > 0.0f ? m_run : -INFINITY;
+          ml[1] = l;
+        } else if (a.lse != nullptr) {
+          a.lse[static_cast<int64_t>(q) * kHeads + h] =
+              l > 0.0f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+      }
+      const int last = ntiles - 1;
+      const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag);
+      good = bar_and(1, 128, got) != 0;
+      if (good) {
         tc_fence_after();
-        const uint64_t kb = kv_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
-        if (elect_one()) {
-#pragma unroll 3
-          for (int kc = 0; kc < 9; ++kc)
+        const int dim_in_tile = warp * 32 + lane;
+#pragma unroll 1
+        for (int d = 0; d < 4; ++d) {
+          const int dim = d * 128 + dim_in_tile;
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tmem + kTmemO + lane_base + d * 64 + half * 32, v);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-              mma_f16(tmem + b * 32, q_desc0 + static_cast<uint64_t>((kc * 8192 + ks * 32) >> 4),
-                      kb + static_cast<uint64_t>((kc * kKVChunk + ks * 32) >> 4), idesc_qk, (kc | ks) != 0);
-          tc_commit(&s_full[b]);
+            for (int i = 0; i < 32; ++i) {
+              const int hh = half * 32 + i;
+              const float o = v[i] * sOutScale[hh];
+              if (split_out) {
+                a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = o;
+              } else {
+                const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
+                if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
+                else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
+              }
+            }
+          }
         }
-        __syncwarp();
-        if (T >= 1 && !issue_pv(T - 1)) { good = false; break; }
       }
-      if (good && !issue_pv(ntiles - 1)) good = false;
-      if (!good && lane == 0) {
-        record_error(a.err, DSA_ERR_TIMEOUT, 10);
-        *abort_flag = 1;
-      }
+    }
+    if (!good && lane == 0) {
+      record_error(a.err, DSA_ERR_TIMEOUT, 13);
+      *abort_flag = 1;
+    }
+    if (!q_landed && tid == 0) wait_drain(q_full, 0);   // the Q copy may still be landing
+    __syncwarp();
+  } else if (ntiles > 0 && warp == kMmaWarp) {
+    // ---------------------------------------------------------------- tcgen05 issuer (whole warp)
+    // Descriptors are formed once and advanced by constants; MMAs and commits come from
+    // one elected lane of the converged warp.
+    const uint32_t idesc_qk = idesc_make(fmt, fmt, false, false, 128, kMlaTile);
+    const uint32_t idesc_pv = idesc_make(fmt, fmt, true, false, 128, 64);
+    const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);                 // K-major view
+    const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);            // MN-major view
+    const uint64_t p_desc0 = sdesc_sw128(smem_u32(sKV + kPChunk * kKVChunk), 16, 1024);
+    bool good = wait_warp(q_ready, 0, abort_flag);
+    tc_fence_after();
+    auto issue_pv = [&](int T) {
+      const int b = T & 1;
+      if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint64_t vb = v_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
+      const uint64_t pb = p_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
       if (elect_one()) {
-        tc_commit(drain);
-        wait_drain(drain, 0);
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+#pragma unroll
+          for (int ks = 0; ks < kMlaTile / 16; ++ks)
+            mma_f16(tmem + kTmemO + d * 64, vb + static_cast<uint64_t>(((2 * d) * kKVChunk + ks * 2048) >> 4),
+                    pb + static_cast<uint64_t>((ks * 32) >> 4), idesc_pv, (T > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(&pv_done[b]);
       }
       __syncwarp();
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ producer
-      // Lane j owns row j of every tile. Its slot comes from the staged list; its five
-      // scales are loaded two tiles ahead into registers, so no global load sits on the
-      // per-tile path.
-      auto slot_of = [&](int T) {
-        const int i = T * kMlaTile + lane;
-        if (T >= ntiles) return -1;
-        if (list_in_smem) return static_cast<int>(sIdxList[i]);
-        int slot = i < nkeys ? phys[k0 + i] : -1;
-        if (slot < -1 || slot >= a.num_slots) {
-          record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(slot));
-          slot = -1;
-        }
-        return slot;
-      };
-      float sc_a[kKvGroups], sc_b[kKvGroups];   // scales of tiles T and T+1
-      auto load_scales = [&](int slot, float (&sc)[kKvGroups]) {
+      return true;
+    };
+    for (int T = 0; T < ntiles && good; ++T) {
+      const int b = T & 1;
+      if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag)) { good = false; break; }
+      if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
+      tc_fence_after();
+      const uint64_t kb = kv_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
+      if (elect_one()) {
+#pragma unroll 3
+        for (int kc = 0; kc < 9; ++kc)
 #pragma unroll
-        for (int g = 0; g < kKvGroups; ++g)
-          sc[g] = (FP8 && slot >= 0) ? a.kv_scale[static_cast<int64_t>(slot) * kKvGroups + g] : 0.0f;
-      };
-      int slot_a = slot_of(0), slot_b = slot_of(1);
-      load_scales(slot_a, sc_a);
-      load_scales(slot_b, sc_b);
-      bool good = true;
-      for (int T = 0; T < ntiles; ++T) {
-        const int st = T % kMlaStages;
-        if (!wait_warp(&stage_empty[st], ((T / kMlaStages) & 1) ^ 1, abort_flag)) { good = false; break; }
-        uint8_t* meta = sStageMeta + st * kStageMetaBytes;
-        uint32_t* mult = reinterpret_cast<uint32_t*>(meta);            // [32][5]
-        int32_t* E = reinterpret_cast<int32_t*>(meta + 640);           // [32]
-        int32_t* slots = reinterpret_cast<int32_t*>(meta + 768);       // [32]
-        const int slot = slot_a;
-        if (FP8 && slot >= 0)
-          bulk_load(sStage + st * kStageRows + lane * kRowBytes, a.kv + static_cast<int64_t>(slot) * kRowBytes,
-                    kRowBytes, &stage_full[st]);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(tmem + b * kMlaTile, q_desc0 + static_cast<uint64_t>((kc * 8192 + ks * 32) >> 4),
+                    kb + static_cast<uint64_t>((kc * kKVChunk + ks * 32) >> 4), idesc_qk, (kc | ks) != 0);
+        tc_commit(&s_full[b]);
+      }
+      __syncwarp();
+      if ((T & 1) && !(issue_pv(T - 1) && issue_pv(T))) { good = false; break; }
+    }
+    if (good && (ntiles & 1) && !issue_pv(ntiles - 1)) good = false;
+    if (!good && lane == 0) {
+      record_error(a.err, DSA_ERR_TIMEOUT, 10);
+      *abort_flag = 1;
+    }
+    // every MMA this warp issued has finished before the CTA frees TMEM
+    if (elect_one()) {
+      tc_commit(drain);
+      wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else if (ntiles > 0 && warp >= kLoadWarp0 && warp < kLoadWarp0 + 6) {
+    // ---------------------------------------------------------------- loaders (two groups)
+    // Piece p of a tile is 16 bytes of row p / R at column byte (p % R) * 16, R = 36 (fp8)
+    // or 72 (bf16) pieces per row; thread t of a group owns pieces t + 96 i. An fp8 tile
+    // is one batch of 24 pieces per thread, loaded a tile pair ahead; a bf16 tile is two
+    // batches, the second loaded when it is needed.
+    const int g = (warp - kLoadWarp0) / 3;
+    const int lt = tid - (kLoadWarp0 + 3 * g) * 32;
+    const int bar_id = 2 + g;
+    constexpr int kRowPieces = FP8 ? 36 : 72;
+    constexpr int kRowBytes = FP8 ? kDimK : 2 * kDimK;
+    constexpr int kBatches = FP8 ? 1 : 2;
+    uint32_t* mult = sGrpMeta + g * (kGrpMetaBytes / 4);
+    KVMeta* km = sKVMeta + g;
+    uint8_t* kv = sKV + g * kKVBytes;
+    uint4 raw[kBatchPieces];
+    float sc[kKvGroups];
+    int my_slot = -1;   // row lt's slot (threads lt < 64)
+    // all slot lookups first, then all loads, so that no lookup waits behind a load
+    auto fetch = [&](int T, int batch) {
+      int sl[kBatchPieces];
+#pragma unroll
+      for (int i = 0; i < kBatchPieces; ++i) {
+        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+        sl[i] = slot_at(T, p / kRowPieces);
+      }
+#pragma unroll
+      for (int i = 0; i < kBatchPieces; ++i) {
+        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+        const int c16 = p % kRowPieces;
+        raw[i] = sl[i] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.kv + static_cast<int64_t>(sl[i]) * kRowBytes) + c16)
+                            : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto fetch_meta = [&](int T) {
+      if (lt < kMlaTile) {
+        my_slot = slot_at(T, lt);
+#pragma unroll
+        for (int k = 0; k < kKvGroups; ++k)
+          sc[k] = (FP8 && my_slot >= 0) ? __ldg(a.kv_scale + static_cast<int64_t>(my_slot) * kKvGroups + k) : 0.0f;
+      }
+    };
+    auto store = [&](int batch) {
+#pragma unroll
+      for (int i = 0; i < kBatchPieces; ++i) {
+        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+        const int row = p / kRowPieces, c16 = p - row * kRowPieces;
+        if (FP8) {
+          const uint32_t mw = mult[row * kKvGroups + (c16 >> 3)];
+          const __half2 m2 = *reinterpret_cast<const __half2*>(&mw);
+          uint4 o0, o1;
+          dequant4_f16(raw[i].x, m2, o0.x, o0.y);
+          dequant4_f16(raw[i].y, m2, o0.z, o0.w);
+          dequant4_f16(raw[i].z, m2, o1.x, o1.y);
+          dequant4_f16(raw[i].w, m2, o1.z, o1.w);
+          uint8_t* blk = kv + (c16 >> 2) * kKVChunk;
+          const int u = (c16 & 3) * 2;
+          // alternate which half goes first by chunk parity: spreads a warp's stores over banks
+          if ((c16 >> 2) & 1) {
+            *reinterpret_cast<uint4*>(blk + swz(row, u + 1)) = o1;
+            *reinterpret_cast<uint4*>(blk + swz(row, u)) = o0;
+          } else {
+            *reinterpret_cast<uint4*>(blk + swz(row, u)) = o0;
+            *reinterpret_cast<uint4*>(blk + swz(row, u + 1)) = o1;
+          }
+        } else {
+          *reinterpret_cast<uint4*>(kv + (c16 >> 3) * kKVChunk + swz(row, c16 & 7)) = raw[i];
+        }
+      }
+    };
+    bool good = true;
+    if (g < ntiles) {
+      fetch_meta(g);
+      fetch(g, 0);
+    }
+    for (int T = g; T < ntiles; T += 2) {
+      // the buffer was last read by PV(T-2)
+      bool ok = T < 2 || wait_warp(&pv_done[g], ((T >> 1) & 1) ^ 1, abort_flag);
+      if (ok && lt < kMlaTile) {
+        // row meta: exponent E_j, multipliers s_g / 2^E_j, validity
         int Ej = 0;
         if (FP8) {
           float smax = 0.0f;
 #pragma unroll
-          for (int g = 0; g < kKvGroups; ++g) smax = fmaxf(smax, sc_a[g]);
+          for (int k = 0; k < kKvGroups; ++k) smax = fmaxf(smax, sc[k]);
           Ej = smax > 0.0f ? float_exponent(smax) : 0;
           const float inv = exp2i(-Ej);
 #pragma unroll
-          for (int g = 0; g < kKvGroups; ++g) {
-            const __half2 m2 = __float2half2_rn(sc_a[g] * inv);
-            mult[lane * kKvGroups + g] = *reinterpret_cast<const uint32_t*>(&m2);
+          for (int k = 0; k < kKvGroups; ++k) {
+            const __half2 m2 = __float2half2_rn(sc[k] * inv);
+            mult[lt * kKvGroups + k] = *reinterpret_cast<const uint32_t*>(&m2);
           }
         }
-        E[lane] = Ej;
-        slots[lane] = slot;
-        const unsigned vm = __ballot_sync(0xffffffffu, slot >= 0);
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&stage_full[st], FP8 ? __popc(vm) * kRowBytes : 0u);
-        // rotate the two-tile lookahead
-        slot_a = slot_b;
-#pragma unroll
-        for (int g = 0; g < kKvGroups; ++g) sc_a[g] = sc_b[g];
-        slot_b = slot_of(T + 2);
-        load_scales(slot_b, sc_b);
-      }
-      if (!good && lane == 0) {
-        record_error(a.err, DSA_ERR_TIMEOUT, 11);
-        *abort_flag = 1;
-      }
-      // bounded drain of this warp's outstanding row copies
-      if (lane == 0 && FP8)
-        for (int T = max(0, ntiles - kMlaStages); T < ntiles; ++T)
-          wait_drain(&stage_full[T % kMlaStages], (T / kMlaStages) & 1);
-      __syncwarp();
-    } else if (warp == 2 || warp == 3) {
-      // ------------------------------------------------------------ dequantisers
-      const int ct = tid - 64;   // 0..63
-      bool good = true;
-      for (int T = 0; T < ntiles; ++T) {
-        const int st = T % kMlaStages, b = T & 1;
-        if (!wait_warp(&stage_full[st], (T / kMlaStages) & 1, abort_flag)) { good = false; break; }
-        if (T >= 2 && !wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
-        const uint8_t* meta = sStageMeta + st * kStageMetaBytes;
-        const uint32_t* mult = reinterpret_cast<const uint32_t*>(meta);
-        const int32_t* slots = reinterpret_cast<const int32_t*>(meta + 768);
-        uint8_t* kv = sKV + b * kKVBytes;
-        if (FP8) {
-          const uint8_t* rows = sStage + st * kStageRows;
-#pragma unroll 3
-          for (int c = ct; c < kMlaTile * 36; c += 64) {
-            const int j = c / 36, cc = c - j * 36;
-            uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-            if (slots[j] >= 0) {
-              const uint4 raw = *reinterpret_cast<const uint4*>(rows + j * kRowBytes + cc * 16);
-              const uint32_t mw = mult[j * kKvGroups + (cc >> 3)];
-              const __half2 m2 = *reinterpret_cast<const __half2*>(&mw);
-              dequant4_f16(raw.x, m2, o0.x, o0.y);
-              dequant4_f16(raw.y, m2, o0.z, o0.w);
-              dequant4_f16(raw.z, m2, o1.x, o1.y);
-              dequant4_f16(raw.w, m2, o1.z, o1.w);
-            }
-            uint8_t* blk = kv + (cc >> 2) * kKVChunk;
-            *reinterpret_cast<uint4*>(blk + swz(j, (cc & 3) * 2)) = o0;
-            *reinterpret_cast<uint4*>(blk + swz(j, (cc & 3) * 2 + 1)) = o1;
-          }
-        } else {
-          for (int c = ct; c < kMlaTile * 72; c += 64) {
-            const int j = c / 72, cc = c - j * 72;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (slots[j] >= 0)
-              v = *reinterpret_cast<const uint4*>(a.kv + static_cast<int64_t>(slots[j]) * (2 * kDimK) + cc * 16);
-            *reinterpret_cast<uint4*>(kv + (cc >> 3) * kKVChunk + swz(j, cc & 7)) = v;
-          }
-        }
-        if (warp == 2) {   // row exponents and validity of this tile, for the softmax warps
-          const int32_t* E = reinterpret_cast<const int32_t*>(meta + 640);
-          int32_t* km = sKVMeta + b * 64;
-          km[lane] = E[lane];
-          const unsigned vm = __ballot_sync(0xffffffffu, slots[lane] >= 0);
-          if (lane == 0) km[32] = static_cast<int32_t>(vm);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
+        const bool valid = my_slot >= 0;
+        km->kmul[lt] = valid ? exp2i(Ej) : 0.0f;
+        km->kadd[lt] = valid ? 0.0f : -INFINITY;
+        km->E[lt] = Ej;
+        const unsigned vm = __ballot_sync(0xffffffffu, valid);
+        const int em = __reduce_max_sync(0xffffffffu, valid ? Ej : kNoExp);
         if (lane == 0) {
-          mbar_arrive(&kv_full[b]);
-          mbar_arrive(&stage_empty[st]);
+          km->vmask[lt >> 5] = vm;
+          km->emax[lt >> 5] = em;
         }
       }
-      if (!good && lane == 0) {
-        record_error(a.err, DSA_ERR_TIMEOUT, 12);
-        *abort_flag = 1;
+      good = bar_and(bar_id, kLoadThreads, ok) != 0;
+      if (!good) break;
+      store(0);
+      if (kBatches > 1) {
+        fetch(T, 1);
+        store(1);
       }
+      fence_proxy_async_smem();
       __syncwarp();
-    } else {
-      // ------------------------------------------------------------ softmax group (warps 4..7)
-      const bool is_sm = warp < 6;            // warps 4,5: heads 0..63 = TMEM lanes 0..63
-      const int quarter = warp & 3;           // TMEM lane quarter this warp may access
-      const int h = (warp - 4) * 32 + lane;   // head (meaningful for warps 4,5)
-      const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-      float m_run = -INFINITY, l_run = 0.0f, cq = 0.0f;
-      int e_ref = kNoExp;                     // running max of the rows' exponents (same in every thread)
-      if (is_sm) cq = sCq[h];
-      bool good = true;
-      for (int T = 0; T < ntiles; ++T) {
-        const int b = T & 1;
-        float y[kMlaTile];
-        int need = 0;
-        if (is_sm) {
-          const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
-                           wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
-          if (got) {
-            tc_fence_after();
-            tmem_ld32(tmem + lane_base + b * 32, y);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[b]);
-            const int32_t* km = sKVMeta + b * 64;
-            const unsigned vm = static_cast<unsigned>(km[32]);
-            float ymax = -INFINITY;
-            int etile = kNoExp;
-#pragma unroll
-            for (int j = 0; j < kMlaTile; ++j) {
-              const bool v = (vm >> j) & 1u;
-              y[j] = v ? y[j] * cq * exp2i(km[j]) : -INFINITY;
-              ymax = fmaxf(ymax, y[j]);
-              if (v) etile = max(etile, km[j]);
-            }
-            float alpha = 1.0f;
-            if (vm != 0u) {
-              if (m_run == -INFINITY) {
-                m_run = ymax;                       // first tile with a valid row: nothing accumulated yet
-              } else if (ymax > m_run + 8.0f) {
-                alpha = exp2f(m_run - ymax);
-                l_run *= alpha;
-                m_run = ymax;
-              }
-              if (e_ref == kNoExp) {
-                e_ref = etile;
-              } else if (etile > e_ref) {
-                alpha *= exp2i(e_ref - etile);
-                e_ref = etile;
-              }
-            }
-            sAlpha[h] = alpha;
-            need = alpha != 1.0f ? 1 : 0;
-          } else {
-            good = false;
-          }
-        }
-        need = group_or(need);
-        good = group_and(good) != 0;
-        if (!good) break;
-        if (need) {
-          // rescale the O^T columns (heads) by alpha; PV(T-1) must have finished first
-          const bool got = wait_warp(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag);
-          if (got) {
-            tc_fence_after();
-#pragma unroll 1
-            for (int d = 0; d < 4; ++d)
-#pragma unroll 1
-              for (int half = 0; half < 2; ++half) {
-                float v[32];
-                const uint32_t addr = tmem_O + lane_base + d * 64 + half * 32;
-                tmem_ld32(addr, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= sAlpha[half * 32 + i];
-                tmem_st32(addr, v);
-              }
-          }
-          good = group_and(got) != 0;
-          if (!good) break;
-        }
-        if (is_sm) {
-          // the P half this tile writes was last read by PV(T-2)
-          const bool got = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag);
-          if (got) {
-            const int32_t* km = sKVMeta + b * 64;
-            uint8_t* prow = sP + h * 128;
-            float lsum = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t w[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = 8 * c + 2 * e;
-                const float p0 = m_run == -INFINITY ? 0.0f : exp2f(y[j] - m_run);
-                const float p1 = m_run == -INFINITY ? 0.0f : exp2f(y[j + 1] - m_run);
-                lsum += p0 + p1;
-                if (FP8) {
-                  const float d0 = exp2i(km[j] - e_ref), d1 = exp2i(km[j + 1] - e_ref);
-                  __half2 hh = __floats2half2_rn(p0 * d0, p1 * d1);
-                  w[e] = *reinterpret_cast<uint32_t*>(&hh);
-                } else {
-                  __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-                  w[e] = *reinterpret_cast<uint32_t*>(&bb);
-                }
-              }
-              *reinterpret_cast<uint4*>(prow + (((b * 4 + c) ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            l_run += lsum;
-            fence_proxy_async_smem();
-          } else {
-            good = false;
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[b]);
-        good = group_and(good) != 0;
-        if (!good) break;
+      if (lane == 0) mbar_arrive(&kv_full[g]);
+      if (T + 2 < ntiles) {
+        fetch_meta(T + 2);
+        fetch(T + 2, 0);
       }
-      // ---- epilogue: warps 4..7 read O^T (lanes = dims), softmax threads supply per-head scales
-      if (good) {
-        const bool split_out = a.nsplit > 1;
-        if (is_sm) {
-          const float l = l_run;
-          const float oscale = exp2i(e_ref == kNoExp ? 0 : e_ref);
-          sOutScale[h] = split_out ? oscale : (l > 0.0f ? oscale / l : 0.0f);
-          if (split_out) {
-            float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * 2;
-            ml[0] = l > 0.0f ? m_run : -INFINITY;
-            ml[1] = l;
-          } else if (a.lse != nullptr) {
-            a.lse[static_cast<int64_t>(q) * kHeads + h] =
-                l > 0.0f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
-          }
-        }
-        const int last = ntiles - 1;
-        const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag);
-        good = group_and(got) != 0;
-        if (good) {
-          tc_fence_after();
-          const int dim_in_tile = quarter * 32 + lane;
-#pragma unroll 1
-          for (int d = 0; d < 4; ++d) {
-            const int dim = d * 128 + dim_in_tile;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-              float v[32];
-              tmem_ld32(tmem_O + lane_base + d * 64 + half * 32, v);
-#pragma unroll 4
-              for (int i = 0; i < 32; ++i) {
-                const int hh = half * 32 + i;
-                const float o = v[i] * sOutScale[hh];
-                if (split_out) {
-                  a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = o;
-                } else {
-                  const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
-                  if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
-                  else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
-                }
-              }
-            }
-          }
-        }
-      }
-      if (!good && lane == 0) {
-        record_error(a.err, DSA_ERR_TIMEOUT, 13);
-        *abort_flag = 1;
-      }
-      __syncwarp();
+      bar_and(bar_id, kLoadThreads, 1);   // the multipliers of tile T are no longer read
     }
+    if (!good && lane == 0) {
+      record_error(a.err, DSA_ERR_TIMEOUT, 12);
+      *abort_flag = 1;
+    }
+    __syncwarp();
   }
 
   if (ntiles == 0) {
@@ -611,15 +641,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       }
     }
   }
-  if (!ok && tid == 0) {
-    record_error(a.err, DSA_ERR_TIMEOUT, 14);
-    wait_drain(q_full, 0);   // the Q copy may still be landing
-  }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, kMlaTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kMlaTmemCols);
 }
 
 // Log-sum-exp merge of the split partials: M = max_s m_s, a_s = 2^(m_s - M),
