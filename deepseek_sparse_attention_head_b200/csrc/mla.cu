@@ -7,17 +7,18 @@
 //
 // Design (sm_100a): grid = (query, split); a CTA walks 64-row tiles of its share of the
 // index list through two tile buffers, with warp-specialised roles:
-//   warps 5-10 loaders, two groups of three: group g fills buffer g with tiles g, g+2, ...
-//             Each thread keeps 24 sixteen-byte pieces of its group's next tile in flight
-//             (plain global loads issued a tile pair ahead), then turns fp8 codes into
+//   warps 5-12 loaders, all on every tile, tiles alternating between the two buffers.
+//             Each thread keeps 9 sixteen-byte pieces of each of the next two tiles in
+//             flight (plain global loads issued two tiles ahead), then turns fp8 codes into
 //             fp16 (exact) x a per-row multiplier s_g / 2^E_j and stores them 128-byte
 //             swizzled: the tile is the K operand of QK (K-major) and the V operand of PV
 //             (MN-major) at once. E_j is the row's power-of-two exponent.
-//   warp 4    tcgen05 issuer: S = Q' K'^T (M=128, rows 64..127 unused, N=64 keys),
+//   warp 4    tcgen05 issuer: S = Q' K'^T (M=64 heads, N=64 keys),
 //             O^T += V'^T P'^T (4 x M=128 dims, N=64 heads); fp32 accumulators in TMEM.
 //             Issue order QK(t), QK(t+1), PV(t), PV(t+1) lets one buffer refill while the
 //             other tile's MMAs run.
-//   warps 0-1 softmax, one thread per head (its TMEM lane): running max with lazy
+//   warps 0-3 softmax, one thread per head (M=64 puts head h in TMEM lane
+//             32 (h / 16) + h % 16, so each warp owns 16 heads): running max with lazy
 //             rescaling (only when a tile's max exceeds it by more than 8 in log2 units),
 //             exact fp32 normaliser, fp16 weights P' = p * 2^(E_j - E_ref) written into
 //             the tile's rope chunk, which QK has finished with.
@@ -34,12 +35,12 @@
 namespace dsa {
 
 constexpr int kMlaTile = 64;
-constexpr int kMlaWarps = 11;
+constexpr int kMlaWarps = 13;
 constexpr int kMlaThreads = kMlaWarps * 32;
 constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp0 = 5;                 // loader group g: warps 5 + 3g .. 7 + 3g
-constexpr int kLoadThreads = 96;              // per group
-constexpr int kBatchPieces = 24;              // 16-byte pieces per loader thread and batch
+constexpr int kLoadWarp0 = 5;                 // loaders: warps 5 .. 12
+constexpr int kLoadThreads = 256;
+constexpr int kBatchPieces = 9;               // 16-byte pieces per loader thread and batch
 constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,128); O^T: cols [128, 384)
 constexpr uint32_t kTmemO = 128;
 constexpr int kNoExp = -100000;               // "no valid row seen yet"
@@ -52,7 +53,7 @@ constexpr int kOffQ = 0;                                        // 9 x [64 x 128
 constexpr int kOffKV = kOffQ + 9 * 8192;                        // 2 x 9 x [64 x 128 B]
 constexpr int kOffKVMeta = kOffKV + 2 * kKVBytes;               // 2 x per-key tables (KVMeta)
 constexpr int kKVMetaBytes = 1152;
-constexpr int kOffGrpMeta = kOffKVMeta + 2 * kKVMetaBytes;      // 2 x mult[64][5] (fp16x2)
+constexpr int kOffGrpMeta = kOffKVMeta + 2 * kKVMetaBytes;      // per buffer: mult[64][5] (fp16x2)
 constexpr int kGrpMetaBytes = kMlaTile * kKvGroups * 4;
 constexpr int kOffHead = kOffGrpMeta + 2 * kGrpMetaBytes;       // cq[64], alpha[64], outscale[64]
 constexpr int kOffBars = kOffHead + 768;
@@ -172,9 +173,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_ready, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 3);
+      mbar_init(&kv_full[i], 8);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 2);
+      mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
       mbar_init(&pv_done[i], 1);
     }
@@ -265,8 +266,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     good = bar_and(1, 128, good) != 0;
 
-    const bool is_sm = warp < 2;            // warps 0,1: heads 0..63 = TMEM lanes 0..63
-    const int h = warp * 32 + lane;         // head (meaningful for warps 0,1)
+    const bool is_sm = lane < 16;           // lanes 0..15 of warp w hold heads 16w .. 16w+15
+    const int h = warp * 16 + (lane & 15);  // (lanes 16..31 mirror them and write nothing)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m_run = -INFINITY, l_run = 0.0f, cq = 0.0f;
     int e_ref = kNoExp;                     // running max of the rows' exponents (same in every thread)
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       KVMeta* km = sKVMeta + b;
       float y[kMlaTile];
       int need = 0;
-      if (is_sm) {
+      {
         const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
                          wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
         if (got) {
@@ -315,9 +316,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             }
           }
           // this thread also owns key h of the tile: its P' factor 2^(E_h - E_ref)
-          km->fac[h] = km->kadd[h] == 0.0f ? exp2i(km->E[h] - e_ref) : 0.0f;
-          sAlpha[h] = alpha;
-          need = alpha != 1.0f ? 1 : 0;
+          if (is_sm) {
+            km->fac[h] = km->kadd[h] == 0.0f ? exp2i(km->E[h] - e_ref) : 0.0f;
+            sAlpha[h] = alpha;
+          }
+          need = (is_sm && alpha != 1.0f) ? 1 : 0;
         } else {
           good = false;
         }
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // ---------------------------------------------------------------- tcgen05 issuer (whole warp)
     // Descriptors are formed once and advanced by constants; MMAs and commits come from
     // one elected lane of the converged warp.
-    const uint32_t idesc_qk = idesc_make(fmt, fmt, false, false, 128, kMlaTile);
+    const uint32_t idesc_qk = idesc_make(fmt, fmt, false, false, 64, kMlaTile);
     const uint32_t idesc_pv = idesc_make(fmt, fmt, true, false, 128, 64);
     const uint64_t q_desc0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);                 // K-major view
@@ -491,26 +494,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       wait_drain(drain, 0);
     }
     __syncwarp();
-  } else if (ntiles > 0 && warp >= kLoadWarp0 && warp < kLoadWarp0 + 6) {
-    // ---------------------------------------------------------------- loaders (two groups)
-    // Piece p of a tile is 16 bytes of row p / R at column byte (p % R) * 16, R = 36 (fp8)
-    // or 72 (bf16) pieces per row; thread t of a group owns pieces t + 96 i. An fp8 tile
-    // is one batch of 24 pieces per thread, loaded a tile pair ahead; a bf16 tile is two
-    // batches, the second loaded when it is needed.
-    const int g = (warp - kLoadWarp0) / 3;
-    const int lt = tid - (kLoadWarp0 + 3 * g) * 32;
-    const int bar_id = 2 + g;
+  } else if (ntiles > 0 && warp >= kLoadWarp0) {
+    // ---------------------------------------------------------------- loaders
+    // All eight loader warps (two per SM sub-partition, which balances the fp8 -> fp16
+    // conversions) work on every tile. Piece p of a tile is 16 bytes of row p / R at column
+    // byte (p % R) * 16, R = 36 (fp8) or 72 (bf16) pieces per row; thread t owns pieces
+    // t + 256 i. Register sets A and B hold the even and the odd tiles: an fp8 tile is one
+    // batch of 9 pieces per thread, loaded two tiles ahead; a bf16 tile is two batches, the
+    // second loaded when it is needed.
+    const int lt = tid - kLoadWarp0 * 32;
     constexpr int kRowPieces = FP8 ? 36 : 72;
     constexpr int kRowBytes = FP8 ? kDimK : 2 * kDimK;
     constexpr int kBatches = FP8 ? 1 : 2;
-    uint32_t* mult = sGrpMeta + g * (kGrpMetaBytes / 4);
-    KVMeta* km = sKVMeta + g;
-    uint8_t* kv = sKV + g * kKVBytes;
-    uint4 raw[kBatchPieces];
-    float sc[kKvGroups];
-    int my_slot = -1;   // row lt's slot (threads lt < 64)
+    uint4 rawA[kBatchPieces], rawB[kBatchPieces];
+    float scA[kKvGroups], scB[kKvGroups];
+    int slotA = -1, slotB = -1;   // row lt's slot (threads lt < 64)
     // all slot lookups first, then all loads, so that no lookup waits behind a load
-    auto fetch = [&](int T, int batch) {
+    auto fetch = [&](uint4 (&raw)[kBatchPieces], int T, int batch) {
       int sl[kBatchPieces];
 #pragma unroll
       for (int i = 0; i < kBatchPieces; ++i) {
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                             : make_uint4(0u, 0u, 0u, 0u);
       }
     };
-    auto fetch_meta = [&](int T) {
+    auto fetch_meta = [&](float (&sc)[kKvGroups], int& my_slot, int T) {
       if (lt < kMlaTile) {
         my_slot = slot_at(T, lt);
 #pragma unroll
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           sc[k] = (FP8 && my_slot >= 0) ? __ldg(a.kv_scale + static_cast<int64_t>(my_slot) * kKvGroups + k) : 0.0f;
       }
     };
-    auto store = [&](int batch) {
+    auto store = [&](const uint4 (&raw)[kBatchPieces], int batch, uint8_t* kv, const uint32_t* mult) {
 #pragma unroll
       for (int i = 0; i < kBatchPieces; ++i) {
         const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
@@ -561,14 +561,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
     };
-    bool good = true;
-    if (g < ntiles) {
-      fetch_meta(g);
-      fetch(g, 0);
-    }
-    for (int T = g; T < ntiles; T += 2) {
+    // one tile: wait for its buffer, publish the row tables, convert, hand over, prefetch T+2
+    auto step = [&](uint4 (&raw)[kBatchPieces], float (&sc)[kKvGroups], int& my_slot, int T) -> bool {
+      const int b = T & 1;
       // the buffer was last read by PV(T-2)
-      bool ok = T < 2 || wait_warp(&pv_done[g], ((T >> 1) & 1) ^ 1, abort_flag);
+      const bool ok = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag);
+      uint32_t* mult = sGrpMeta + b * (kGrpMetaBytes / 4);
+      KVMeta* km = sKVMeta + b;
       if (ok && lt < kMlaTile) {
         // row meta: exponent E_j, multipliers s_g / 2^E_j, validity
         int Ej = 0;
@@ -595,21 +594,33 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           km->emax[lt >> 5] = em;
         }
       }
-      good = bar_and(bar_id, kLoadThreads, ok) != 0;
-      if (!good) break;
-      store(0);
+      // also orders this tile's table writes after every loader's reads of tile T-2's
+      if (!bar_and(2, kLoadThreads, ok)) return false;
+      uint8_t* kv = sKV + b * kKVBytes;
+      store(raw, 0, kv, mult);
       if (kBatches > 1) {
-        fetch(T, 1);
-        store(1);
+        fetch(raw, T, 1);
+        store(raw, 1, kv, mult);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&kv_full[g]);
+      if (lane == 0) mbar_arrive(&kv_full[b]);
       if (T + 2 < ntiles) {
-        fetch_meta(T + 2);
-        fetch(T + 2, 0);
+        fetch_meta(sc, my_slot, T + 2);
+        fetch(raw, T + 2, 0);
       }
-      bar_and(bar_id, kLoadThreads, 1);   // the multipliers of tile T are no longer read
+      return true;
+    };
+    fetch_meta(scA, slotA, 0);
+    fetch(rawA, 0, 0);
+    if (ntiles > 1) {
+      fetch_meta(scB, slotB, 1);
+      fetch(rawB, 1, 0);
+    }
+    bool good = true;
+    for (int T = 0; T < ntiles && good; T += 2) {
+      good = step(rawA, scA, slotA, T);
+      if (good && T + 1 < ntiles) good = step(rawB, scB, slotB, T + 1);
     }
     if (!good && lane == 0) {
       record_error(a.err, DSA_ERR_TIMEOUT, 12);
