@@ -266,38 +266,53 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     good = bar_and(1, 128, good) != 0;
 
-    const bool is_sm = lane < 16;           // lanes 0..15 of warp w hold heads 16w .. 16w+15
-    const int h = warp * 16 + (lane & 15);  // (lanes 16..31 mirror them and write nothing)
+    // M=64 puts head h in TMEM lane 32 (h / 16) + h % 16: lanes 0..15 of warp w hold heads
+    // 16w .. 16w+15. Lane l < 16 takes keys 0..31 of its head, lane l + 16 keys 32..63 of
+    // the same head (handed over by shuffle); both keep identical running statistics.
+    const bool is_sm = lane < 16;           // the lane that writes per-head state
+    const int h = warp * 16 + (lane & 15);
+    const int jb = lane < 16 ? 0 : 32;      // this lane's keys: jb .. jb+31
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    float m_run = -INFINITY, l_run = 0.0f, cq = 0.0f;
+    float m_run = -INFINITY, l_run = 0.0f;
     int e_ref = kNoExp;                     // running max of the rows' exponents (same in every thread)
-    if (is_sm) cq = sCq[h];
+    const float cq = sCq[h];
     for (int T = 0; T < ntiles && good; ++T) {
       const int b = T & 1;
       KVMeta* km = sKVMeta + b;
-      float y[kMlaTile];
+      float y[32];
       int need = 0;
       {
         const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
                          wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
         if (got) {
           tc_fence_after();
-          tmem_ld64(tmem + lane_base + b * kMlaTile, y);
+          tmem_ld32(tmem + lane_base + b * kMlaTile + 32, y);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = __shfl_sync(0xffffffffu, y[i], lane & 15);
+          {
+            float y0[32];
+            tmem_ld32(tmem + lane_base + b * kMlaTile, y0);
+            if (is_sm) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) y[i] = y0[i];
+            }
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[b]);
           // logits in log2 units: z = acc * cq * 2^E_j, -inf for unused rows
           float ymax = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < kMlaTile; j += 4) {
-            const float4 mu = *reinterpret_cast<const float4*>(&km->kmul[j]);
-            const float4 ad = *reinterpret_cast<const float4*>(&km->kadd[j]);
+          for (int j = 0; j < 32; j += 4) {
+            const float4 mu = *reinterpret_cast<const float4*>(&km->kmul[jb + j]);
+            const float4 ad = *reinterpret_cast<const float4*>(&km->kadd[jb + j]);
             y[j + 0] = fmaf(y[j + 0], cq * mu.x, ad.x);
             y[j + 1] = fmaf(y[j + 1], cq * mu.y, ad.y);
             y[j + 2] = fmaf(y[j + 2], cq * mu.z, ad.z);
             y[j + 3] = fmaf(y[j + 3], cq * mu.w, ad.w);
             ymax = fmaxf(fmaxf(ymax, fmaxf(y[j + 0], y[j + 1])), fmaxf(y[j + 2], y[j + 3]));
           }
+          ymax = fmaxf(ymax, __shfl_xor_sync(0xffffffffu, ymax, 16));
           const int etile = max(km->emax[0], km->emax[1]);
           float alpha = 1.0f;
           if ((km->vmask[0] | km->vmask[1]) != 0u) {
@@ -315,8 +330,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
               e_ref = etile;
             }
           }
-          // this thread also owns key h of the tile: its P' factor 2^(E_h - E_ref)
           if (is_sm) {
+            // this lane also owns key h of the tile: its P' factor 2^(E_h - E_ref)
             km->fac[h] = km->kadd[h] == 0.0f ? exp2i(km->E[h] - e_ref) : 0.0f;
             sAlpha[h] = alpha;
           }
@@ -348,16 +363,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         good = bar_and(1, 128, got) != 0;
         if (!good) break;
       }
-      if (is_sm) {
+      {
         // p = 2^(z - m) (fp32, summed exactly into l); P' = p * 2^(E_j - E_ref) in the
-        // tile's rope chunk (K-major rows of 64 keys per head)
+        // tile's rope chunk (K-major rows of 64 keys per head; this lane writes 32 of them)
         uint8_t* prow = sKV + b * kKVBytes + kPChunk * kKVChunk + h * 128;
         const float mm = m_run == -INFINITY ? 0.0f : m_run;
         float lsum0 = 0.0f, lsum1 = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 f0 = *reinterpret_cast<const float4*>(&km->fac[8 * c]);
-          const float4 f1 = *reinterpret_cast<const float4*>(&km->fac[8 * c + 4]);
+        for (int c = 0; c < 4; ++c) {
+          const float4 f0 = *reinterpret_cast<const float4*>(&km->fac[jb + 8 * c]);
+          const float4 f1 = *reinterpret_cast<const float4*>(&km->fac[jb + 8 * c + 4]);
           const float fa[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
           uint32_t w[4];
 #pragma unroll
@@ -375,7 +390,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
               w[e] = *reinterpret_cast<uint32_t*>(&bb);
             }
           }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const int unit = (jb >> 3) + c;
+          *reinterpret_cast<uint4*>(prow + ((unit ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         l_run += lsum0 + lsum1;
         fence_proxy_async_smem();
@@ -384,6 +400,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
     }
+    // the two lanes of a head hold halves of its normaliser
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
     // ---- epilogue: warps 0..3 read O^T (lanes = dims), softmax threads supply per-head scales
     if (good) {
       const bool split_out = a.nsplit > 1;
