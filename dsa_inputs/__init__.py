@@ -308,6 +308,12 @@ def algorithmic_bytes(case: dict) -> dict:
                 total=idx_bytes + mla_bytes + q_bytes)
 
 
+def indexer_flops(case: dict) -> int:
+    """Multiply-adds x 2 of the indexer contraction: 64 heads x 128 dims per visible
+    (query, token) pair."""
+    return int(2 * H * DI * int(vis_lengths(case).astype(np.int64).sum()))
+
+
 def to_torch(case: dict, device="cuda") -> dict:
     """Host numpy arrays -> torch tensors on `device` (bf16 bits become torch.bfloat16,
     E4M3 codes become torch.float8_e4m3fn). Plumbing only."""
