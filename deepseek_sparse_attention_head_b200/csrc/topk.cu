@@ -2,12 +2,18 @@
 // transform ("GLM-52 Runs on RTX 4090", kernel list item 2; glm-5.2-4090 README,
 // usage: SGLANG_NSA_FUSE_TOPK=1 fuses the page-mapping transform into top-k).
 //
-// One CTA per query. Scores are mapped to order-preserving 32-bit keys and the
-// k-th largest key is found exactly by a three-digit radix select (12 + 12 + 8 bits)
-// over shared-memory histograms; a last pass emits every key above it plus the
-// needed number of keys equal to it, and maps each logical token through the
-// block table to its physical slot. A query that sees no more than top_k tokens
-// takes all of them (the dense path).
+// One CTA per query. Scores are mapped to order-preserving 32-bit keys.
+//  1. A threshold is estimated from 256 evenly spaced samples of the row, low enough
+//     that about 1.25 k / vis of the samples (plus a margin) lie above it.
+//  2. One pass over the row gathers every key at or above the threshold into shared
+//     memory (per-thread counts, a warp prefix sum and one shared atomic per warp for
+//     every 16K keys).
+//  3. The k-th largest candidate is found exactly by a radix select over the
+//     candidates' offsets from the threshold (12-bit digits, shared-memory
+//     histograms), and the winners are emitted with their physical slots.
+// When the estimate misses (fewer than k candidates, or more than fit), a
+// three-digit radix select over the whole row (12 + 12 + 8 bits) decides instead.
+// A query that sees no more than top_k tokens takes all of them (the dense path).
 #include "kernels.cuh"
 
 namespace dsa {
@@ -20,14 +26,14 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kHistBins = 4096;
-constexpr int kCand = 6144;   // candidates kept in shared memory after the first digit
+constexpr int kCand = 12288;  // candidates kept in shared memory
 
 struct TopkSmem {
   uint32_t hist[kHistBins];
   uint32_t cand_key[kCand];
   int32_t cand_idx[kCand];
   uint32_t wsum[32];
-  uint32_t sel_bin, sel_rem, n_cand, cnt_out, cnt_eq;
+  uint32_t sel_bin, sel_rem, n_cand, cnt_out, cnt_eq, thr, rmax;
 };
 
 // Visits keys[0..n) of a row with 16-byte loads (4 in flight per thread) where the
@@ -80,8 +86,19 @@ __device__ __forceinline__ void select_bin(TopkSmem& sm, uint32_t remaining) {
   }
   if (lane == 0) sm.wsum[warp] = v;
   __syncthreads();
-  uint32_t above = v - mine;
-  for (int w = warp + 1; w < 32; ++w) above += sm.wsum[w];
+  if (warp == 0) {   // suffix sums over the warps: wsum[w] <- sum of warps w+1 .. 31
+    const uint32_t x = sm.wsum[lane];
+    uint32_t y = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t n = __shfl_down_sync(0xffffffffu, y, off);
+      if (lane + off < 32) y += n;
+    }
+    __syncwarp();
+    sm.wsum[lane] = y - x;
+  }
+  __syncthreads();
+  uint32_t above = v - mine + sm.wsum[warp];
   const uint32_t cs[4] = {c0, c1, c2, c3};
 #pragma unroll
   for (int i = 3; i >= 0; --i) {
@@ -92,6 +109,23 @@ __device__ __forceinline__ void select_bin(TopkSmem& sm, uint32_t remaining) {
     above += cs[i];
   }
   __syncthreads();
+}
+
+// Reserves `n` consecutive slots of a shared counter for each lane of a converged, full
+// warp with one atomic per warp; returns the lane's first slot.
+__device__ __forceinline__ uint32_t warp_reserve(uint32_t* counter, uint32_t n) {
+  const int lane = static_cast<int>(threadIdx.x & 31);
+  uint32_t incl = n;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+  uint32_t base = 0;
+  if (lane == 31 && total != 0u) base = atomicAdd(counter, total);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  return base + incl - n;
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkArgs a) {
@@ -124,7 +158,177 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
 
   const float* row = a.scores + static_cast<int64_t>(q) * a.L_max;
 
-  // ---- digit 1 (key bits 31..20) over the whole row
+  // The sampled path needs 16-byte aligned rows (always true for the fused layer, whose
+  // row stride is a multiple of 64); other rows take the whole-row radix select below.
+  const bool aligned_row = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  if (aligned_row) {
+  // ---- 1. threshold from 256 evenly spaced samples (kept in the histogram area)
+  constexpr int kSamples = 256;
+  uint32_t* samp = sm.hist;
+  uint32_t mykey = 0u;
+  if (tid < kSamples) {
+    mykey = order_key(row[static_cast<int>((static_cast<int64_t>(tid) * vis) / kSamples)]);
+    samp[tid] = mykey;
+  }
+  if (tid == 0) {
+    sm.thr = 0u;
+    sm.rmax = 0u;
+    sm.n_cand = 0;
+    sm.cnt_out = 0;
+    sm.cnt_eq = 0;
+  }
+  __syncthreads();
+  if (tid < kSamples) {
+    uint32_t above = 0;      // samples strictly above this thread's sample
+    const uint4* s4 = reinterpret_cast<const uint4*>(samp);
+#pragma unroll 8
+    for (int i = 0; i < kSamples / 4; ++i) {
+      const uint4 v = s4[i];
+      above += (v.x > mykey) + (v.y > mykey) + (v.z > mykey) + (v.w > mykey);
+    }
+    const float expect = static_cast<float>(kSamples) * static_cast<float>(K) / static_cast<float>(vis);
+    const uint32_t need = static_cast<uint32_t>(fminf(1.25f * expect + 3.0f * sqrtf(expect) + 4.0f, 1e9f));
+    // the largest sample with at least `need` samples above it
+    const uint32_t cand = above >= need ? mykey : 0u;
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, cand);
+    if ((tid & 31) == 0 && wmax != 0u) atomicMax(&sm.thr, wmax);
+  }
+  __syncthreads();
+  const uint32_t thr = sm.thr;
+
+  // ---- 2. gather every key >= thr (coalesced, convergent; ballot compaction)
+  {
+    // Batches of 16 keys per thread (four 16-byte loads, coalesced across the block); the
+    // next batch is loaded before this one is processed. One slot reservation per warp and
+    // batch. The row start is 16-byte aligned (the row stride is a multiple of 64 floats).
+    constexpr int kU = 16;
+    constexpr int kBatch = kU * kTopkThreads;
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+    auto load_batch = [&](int base, float4 (&v)[kU / 4]) {
+#pragma unroll
+      for (int j = 0; j < kU / 4; ++j) {
+        const int s_ = base + 4 * (j * kTopkThreads + tid);
+        v[j] = s_ + 3 < vis ? __ldg(r4 + (s_ >> 2))
+                            : make_float4(s_ < vis ? row[s_] : 0.0f, s_ + 1 < vis ? row[s_ + 1] : 0.0f,
+                                          s_ + 2 < vis ? row[s_ + 2] : 0.0f, 0.0f);
+      }
+    };
+    uint32_t lmax = 0;
+    float4 cur[kU / 4], nxt[kU / 4];
+    load_batch(0, cur);
+    for (int base = 0; base < vis; base += kBatch) {
+      if (base + kBatch < vis) load_batch(base + kBatch, nxt);
+      uint32_t takes = 0;
+#pragma unroll
+      for (int j = 0; j < kU / 4; ++j) {
+        const int s_ = base + 4 * (j * kTopkThreads + tid);
+        const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          if (s_ + t < vis && order_key(e[t]) >= thr) takes |= 1u << (4 * j + t);
+      }
+      uint32_t c = warp_reserve(&sm.n_cand, static_cast<uint32_t>(__popc(takes)));
+#pragma unroll
+      for (int j = 0; j < kU / 4; ++j) {
+        const int s_ = base + 4 * (j * kTopkThreads + tid);
+        const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          if (takes & (1u << (4 * j + t))) {
+            const uint32_t u = order_key(e[t]);
+            if (c < static_cast<uint32_t>(kCand)) {
+              sm.cand_key[c] = u;
+              sm.cand_idx[c] = s_ + t;
+            }
+            ++c;
+            lmax = max(lmax, u - thr);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kU / 4; ++j) cur[j] = nxt[j];
+    }
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, lmax);
+    if ((tid & 31) == 0) atomicMax(&sm.rmax, wmax);
+  }
+  __syncthreads();
+  const uint32_t n_c = sm.n_cand;
+  if (n_c >= static_cast<uint32_t>(K) && n_c <= static_cast<uint32_t>(kCand)) {
+    // ---- 3. exact radix select over r = key - thr among the candidates
+    const uint32_t rmax = sm.rmax;
+    int hi = rmax == 0u ? 0 : 32 - __clz(rmax);          // r fits in bits [0, hi)
+    uint32_t prefix = 0u, pmask = 0u, remaining = static_cast<uint32_t>(K);
+#pragma unroll 1
+    while (true) {
+      const int lo_bit = hi > 12 ? hi - 12 : 0;
+      const uint32_t dm = (1u << (hi - lo_bit)) - 1u;      // hi - lo_bit in [0, 12]
+      for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
+      __syncthreads();
+      for (int c = tid; c < static_cast<int>(n_c); c += kTopkThreads) {
+        const uint32_t r = sm.cand_key[c] - thr;
+        if ((r & pmask) == prefix) atomicAdd(&sm.hist[(r >> lo_bit) & dm], 1u);
+      }
+      __syncthreads();
+      select_bin(sm, remaining);
+      prefix |= sm.sel_bin << lo_bit;
+      pmask |= dm << lo_bit;
+      remaining = sm.sel_rem;
+      if (lo_bit == 0) break;
+      hi = lo_bit;
+    }
+    const uint32_t kth = prefix, take_eq = remaining;
+    const uint32_t n_gt = static_cast<uint32_t>(K) - take_eq;
+    // emit: each thread takes candidates tid, tid + 1024, ... (at most kCand / 1024)
+    constexpr int kPer = kCand / kTopkThreads;
+    uint32_t gts = 0, eqs = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int c = j * kTopkThreads + tid;
+      if (c < static_cast<int>(n_c)) {
+        const uint32_t r = sm.cand_key[c] - thr;
+        if (r > kth) gts |= 1u << j;
+        else if (r == kth) eqs |= 1u << j;
+      }
+    }
+    uint32_t pg = warp_reserve(&sm.cnt_out, static_cast<uint32_t>(__popc(gts)));
+    uint32_t pe = warp_reserve(&sm.cnt_eq, static_cast<uint32_t>(__popc(eqs)));
+    // output positions and tokens first, then all block-table lookups, then the stores
+    int pos[kPer], tok[kPer], page[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      pos[j] = -1;
+      tok[j] = 0;
+      const int c = j * kTopkThreads + tid;
+      if (gts & (1u << j)) {
+        if (pg < n_gt) { pos[j] = static_cast<int>(pg); tok[j] = sm.cand_idx[c]; }
+        ++pg;
+      } else if (eqs & (1u << j)) {
+        if (pe < take_eq) { pos[j] = static_cast<int>(n_gt + pe); tok[j] = sm.cand_idx[c]; }
+        ++pe;
+      }
+    }
+    const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_pages;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) page[j] = (po != nullptr && pos[j] >= 0) ? __ldg(bt_row + (tok[j] >> 6)) : 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (page[j] < 0 || page[j] >= a.num_pages) {
+        if (pos[j] >= 0) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(page[j]));
+        page[j] = 0;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (pos[j] < 0) continue;
+      if (lo) lo[pos[j]] = tok[j];
+      if (po) po[pos[j]] = page[j] * kPage + (tok[j] & 63);
+    }
+    return;
+  }
+  __syncthreads();
+  }   // aligned_row
+
+  // ---- fallback: digit 1 (key bits 31..20) over the whole row
   for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
   if (tid == 0) {
     sm.n_cand = 0;

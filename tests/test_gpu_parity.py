@@ -170,3 +170,18 @@ def test_topk_extreme_values():
     assert err == 0
     for i in range(3):
         check_topk_exact(lo[i], base[i], vis[i], 300)
+
+
+def test_topk_unaligned_rows():
+    """A row stride that is not a multiple of 4 floats leaves rows unaligned for 16-byte
+    loads; those rows take the whole-row radix path and must select the same sets."""
+    rng = np.random.default_rng(5)
+    L = 4099
+    scores = rng.standard_normal((3, L)).astype(np.float32)
+    scores[1, ::97] += 4.0
+    vis = np.array([L, L - 3, 3000])
+    case, lo, ph, err = _topk_on_scores(scores, vis, 512)
+    assert err == 0
+    for i in range(3):
+        check_topk_exact(lo[i], scores[i], vis[i], 512)
+    assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
