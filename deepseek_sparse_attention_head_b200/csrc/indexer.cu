@@ -3,40 +3,51 @@
 //
 //   score[q, s] = k_scale[slot(s)] * sum_h (w[q,h] * q_scale[q,h]) * ReLU(<q8[q,h], k8[slot(s)]>)
 //
-// Design (sm_100a): one persistent CTA per SM walks a contiguous range of 256-token
-// tiles (four 64-token pages) of the paged key cache.
+// Design (sm_100a): one persistent CTA per SM walks a contiguous range of tiles of the
+// paged key cache: 512 tokens (eight 64-token pages, 64 KB) for fp8 decode, 256 tokens
+// otherwise.
 //   warp 0     TMA producer: one 64 x 128 B box per page, straight from the block table
-//              (fetched a batch ahead), 128-byte swizzled, into a 4-deep ring of 32 KB
-//              stages; query tiles into their own ring.
+//              (fetched a batch ahead), 128-byte swizzled, into a ring of stages (192 KB of
+//              keys in flight for fp8 decode); query tiles into their own ring.
 //   warp 1     tcgen05 issuer: per 128-token half, D[128 tokens, 64*g heads] =
 //              K_half x Q_group^T, fp8 x fp8 (kind::f8f6f4) or bf16 x bf16 (kind::f16),
-//              fp32 in a ring of TMEM accumulators; MMAs come from an elected lane.
-//   warps 2-9  epilogue, two groups of four taking alternate accumulators: one thread
-//              per token (its TMEM lane) applies ReLU, the head weights and the key scale
-//              (loaded two tiles ahead) and writes the fp32 score.
-// Every synchronisation step costs a few hundred nanoseconds, so a tile carries 33 KB of
-// keys to keep that cost per byte low. Decode (n_q = 1) loads a row's query once per
+//              fp32 in a ring of TMEM accumulator units (two halves per unit for decode,
+//              so one commit and one wait cover 256 tokens); MMAs come from an elected lane.
+//   warps 2-9  epilogue, two groups of four taking alternate units: one thread per token
+//              (its TMEM lane) applies ReLU, the head weights and the key scale (loaded two
+//              tiles ahead) and writes the fp32 score.
+// Every synchronisation step costs a few hundred nanoseconds, so tiles and units are large
+// enough to keep that cost per byte low. Decode (n_q = 1) loads a row's query once per
 // row; chunked prefill streams groups of up to 4 queries (N = 256) past every key tile.
 #include "kernels.cuh"
 
 namespace dsa {
 
-constexpr int kTileTok = 256;
-constexpr int kPagesPerTile = kTileTok / kPage;
-constexpr int kQGroup = 4;
-constexpr int kBatch = 32 / kPagesPerTile;   // tiles whose block-table entries the producer fetches at once
 constexpr int kEpiWarps = 8;                 // two groups of four, alternating accumulators
 constexpr int kIdxThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kIdxTmemCols = 512;       // accumulators of 64 * min(n_q, 4) columns each
 
-template <int KC>
+// KC: 128-byte K-chunks per row (1 = fp8, 2 = bf16). QG: queries per group (1 for decode,
+// 4 for chunked prefill). Decode needs only one query per group, so its query slots and
+// head-weight buffers are small and the key ring holds 192 KB: about what page streaming
+// needs in flight per SM to approach the copy rate.
+template <int KC, int QG>
 struct IdxCfg {
+  // fp8 decode walks 512-token tiles (eight pages, 64 KB) so that the per-tile barrier work
+  // of the tcgen05 issuer is paid per 64 KB; the other forms use 256-token tiles.
+  static constexpr int kTileTok = (KC == 1 && QG == 1) ? 512 : 256;
+  static constexpr int kPagesPerTile = kTileTok / kPage;
+  static constexpr int kBatch = 32 / kPagesPerTile;   // tiles whose block-table entries the producer fetches at once
+  static constexpr int kHalves = kTileTok / 128;       // 128-token MMA halves (M = 128) per tile
+  static constexpr int kUnitHalves = QG == 1 ? 2 : 1;  // halves per accumulator unit (one commit, one wait)
   static constexpr int kChunk = kTileTok * 128;        // one 128-byte K-chunk of a tile
-  static constexpr int kStages = KC == 1 ? 4 : 2;
-  static constexpr int kBSlots = KC == 1 ? 2 : 1;
+  static constexpr int kStages = KC == 1 ? (QG == 1 ? 3 : 4) : 2;
+  static constexpr int kBSlots = (KC == 2 && QG == 4) ? 1 : 2;
   static constexpr int kAStage = KC * kChunk;          // 256 tokens x 128 B per K-chunk
-  static constexpr int kBSlot = KC * 32768;            // 4 queries x 64 heads x 128 B per K-chunk
-  static constexpr int kWBytes = kEpiWarps * 2 * 256 * 4;  // per-warp double-buffered head weights
+  static constexpr int kQChunk = QG * 8192;            // QG queries x 64 heads x 128 B
+  static constexpr int kBSlot = KC * kQChunk;
+  static constexpr int kWPer = kHeads * QG;            // head weights of one query group
+  static constexpr int kWBytes = kEpiWarps * 2 * kWPer * 4;  // per-warp double-buffered head weights
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kAStage;
   static constexpr int kOffW = kOffB + kBSlots * kBSlot;
@@ -46,7 +57,13 @@ struct IdxCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
 };
-static_assert(IdxCfg<1>::kSmem <= 232448 && IdxCfg<2>::kSmem <= 232448, "shared memory");
+static_assert(IdxCfg<1, 1>::kHalves / IdxCfg<1, 1>::kUnitHalves == 2 &&
+                  IdxCfg<1, 4>::kHalves / IdxCfg<1, 4>::kUnitHalves == 2 &&
+                  IdxCfg<2, 1>::kHalves / IdxCfg<2, 1>::kUnitHalves == 1,
+              "units per tile");
+static_assert(IdxCfg<1, 1>::kSmem <= 232448 && IdxCfg<1, 4>::kSmem <= 232448 && IdxCfg<2, 1>::kSmem <= 232448 &&
+                  IdxCfg<2, 4>::kSmem <= 232448,
+              "shared memory");
 
 // Walks the CTA's contiguous range of global tile ids, yielding (row, tile-in-row) and
 // the row's clamped length. Row bounds and lengths live in registers and are reloaded
@@ -89,20 +106,26 @@ struct TileWalker {
 };
 
 // A query group contributes to a tile when one of its queries sees a token of it.
+template <int QG>
 __device__ __forceinline__ bool group_active(const IndexerArgs& a, int b, int g, int tok0, int L) {
   if (a.q_pos == nullptr) return true;
-  const int q0 = b * a.n_q + g * kQGroup;
-  const int nqg = min(kQGroup, a.n_q - g * kQGroup);
+  const int q0 = b * a.n_q + g * QG;
+  const int nqg = min(QG, a.n_q - g * QG);
   for (int j = 0; j < nqg; ++j)
     if (query_vis(a.q_pos, q0 + j, L) > tok0) return true;
   return false;
 }
 
-template <int KC>
+template <int KC, int QG>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                    const IndexerArgs a) {
-  using C = IdxCfg<KC>;
+  using C = IdxCfg<KC, QG>;
+  constexpr int kTileTok = C::kTileTok;
+  constexpr int kPagesPerTile = C::kPagesPerTile;
+  constexpr int kBatch = C::kBatch;
+  constexpr int UH = C::kUnitHalves;
+  constexpr int kUnitsPerTile = C::kHalves / UH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + C::kOffA;
@@ -122,8 +145,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // accumulator ring: 64 columns per query of a group; decode (n_q = 1) gets 8 of them
-  const int acc_cols = kHeads * min(a.n_q, kQGroup);
-  const int n_acc = min(C::kMaxAcc, static_cast<int>(kIdxTmemCols) / acc_cols);
+  const int acc_cols = kHeads * min(a.n_q, QG);        // one 128-token half
+  const int unit_cols = UH * acc_cols;
+  const int n_acc = min(C::kMaxAcc, static_cast<int>(kIdxTmemCols) / unit_cols);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -155,7 +179,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
   const int t_begin = min(total, static_cast<int>(blockIdx.x) * per);
   const int t_end = min(total, t_begin + per);
-  const int ngroups = (a.n_q + kQGroup - 1) / kQGroup;
+  const int ngroups = (a.n_q + QG - 1) / QG;
 
   if (t_begin < t_end) {
     TileWalker walk;
@@ -216,10 +240,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           ++it;
           const int tok0 = t * kTileTok;
           for (int g = 0; g < ngroups; ++g) {
-            if (!group_active(a, b, g, tok0, L)) continue;
-            const int q0 = b * a.n_q + g * kQGroup;
+            if (!group_active<QG>(a, b, g, tok0, L)) continue;
+            const int q0 = b * a.n_q + g * QG;
             if (q0 == cur_q0) continue;
-            const int nqg = min(kQGroup, a.n_q - g * kQGroup);
+            const int nqg = min(QG, a.n_q - g * QG);
             ++bit;
             const int bs = bit % C::kBSlots;
             if (!wait_warp(&b_empty[bs], ((bit / C::kBSlots) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -228,7 +252,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               for (int j = 0; j < nqg; ++j)
 #pragma unroll
                 for (int kc = 0; kc < KC; ++kc)
-                  tma_load_2d(sB + bs * C::kBSlot + kc * 32768 + j * 8192, &tmap_q, kc * 64, (q0 + j) * kHeads,
+                  tma_load_2d(sB + bs * C::kBSlot + kc * C::kQChunk + j * 8192, &tmap_q, kc * 64, (q0 + j) * kHeads,
                               &b_full[bs]);
             }
             cur_q0 = q0;
@@ -264,9 +288,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int tok0 = t * kTileTok;
         const uint64_t ad = a_desc0 + static_cast<uint64_t>((s * C::kAStage) >> 4);
         for (int g = 0; g < ngroups && ok; ++g) {
-          if (!group_active(a, b, g, tok0, L)) continue;
-          const int q0 = b * a.n_q + g * kQGroup;
-          const int nqg = min(kQGroup, a.n_q - g * kQGroup);
+          if (!group_active<QG>(a, b, g, tok0, L)) continue;
+          const int q0 = b * a.n_q + g * QG;
+          const int nqg = min(QG, a.n_q - g * QG);
           if (q0 != cur_q0) {
             if (bit >= 0) {
               if (elect_one()) tc_commit(&b_empty[bit % C::kBSlots]);
@@ -279,21 +303,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
           const uint32_t idesc = idesc_make(fmt, fmt, false, false, 128, kHeads * nqg);
           const uint64_t bd = b_desc0 + static_cast<uint64_t>(((bit % C::kBSlots) * C::kBSlot) >> 4);
-          for (int h2 = 0; h2 < 2; ++h2, ++unit) {
+          for (int u = 0; u < kUnitsPerTile; ++u, ++unit) {
             const int ab = unit % n_acc;
             if (!wait_warp(&acc_empty[ab], ((unit / n_acc) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d = tmem + static_cast<uint32_t>(ab * acc_cols);
             if (elect_one()) {
 #pragma unroll
-              for (int kc = 0; kc < KC; ++kc)
+              for (int hh = 0; hh < UH; ++hh) {
+                const int h2 = u * UH + hh;
+                const uint32_t d = tmem + static_cast<uint32_t>(ab * unit_cols + hh * acc_cols);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                  const uint64_t ao = ad + static_cast<uint64_t>((kc * C::kChunk + h2 * 16384 + ks * 32) >> 4);
-                  const uint64_t bo = bd + static_cast<uint64_t>((kc * 32768 + ks * 32) >> 4);
-                  if (KC == 1) mma_f8(d, ao, bo, idesc, (kc | ks) != 0);
-                  else mma_f16(d, ao, bo, idesc, (kc | ks) != 0);
-                }
+                for (int kc = 0; kc < KC; ++kc)
+#pragma unroll
+                  for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ao = ad + static_cast<uint64_t>((kc * C::kChunk + h2 * 16384 + ks * 32) >> 4);
+                    const uint64_t bo = bd + static_cast<uint64_t>((kc * C::kQChunk + ks * 32) >> 4);
+                    if (KC == 1) mma_f8(d, ao, bo, idesc, (kc | ks) != 0);
+                    else mma_f16(d, ao, bo, idesc, (kc | ks) != 0);
+                  }
+              }
               tc_commit(&acc_full[ab]);
             }
             __syncwarp();
@@ -316,54 +344,67 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       __syncwarp();
     } else {
       // ------------------------------------------------------------ epilogue (warps 2..9)
-      // Two groups of four warps take alternate accumulator units (a unit = a 128-token half
-      // of a tile for one query group); in a group, warp w reads TMEM lanes
-      // [32*(w%4), 32*(w%4)+32), one token per thread. Each thread loads the key scales of
-      // its two tokens of a tile two tiles ahead, from block-table entries loaded four tiles
-      // ahead, so neither load stalls the tile it is used in.
+      // Two groups of four warps take alternate accumulator units (a unit = UH 128-token
+      // halves of a tile for one query group); in a group, warp w reads TMEM lanes
+      // [32*(w%4), 32*(w%4)+32), one token of every half per thread. Each thread loads the
+      // key scales of its tokens of a tile two tiles ahead, from block-table entries
+      // loaded four tiles ahead, so neither load stalls the tile it is used in.
+      constexpr int H = C::kHalves;
       const int eg = (warp - 2) >> 2;
       const int quarter = warp & 3;
       const int row_in_half = quarter * 32 + lane;
-      float* wmine = sW + (warp - 2) * 512;    // two 256-entry buffers per warp
+      const int off = row_in_half & 63;
+      float* wmine = sW + (warp - 2) * 2 * C::kWPer;   // two buffers of one group's weights per warp
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
       int unit = 0, cur_q0 = -1, wb = 1;
       bool ok = true;
       TileWalker w2 = walk, w4 = walk;
-      // page of this thread's token in half h of the next tile of walker w (-1 past the end)
-      auto tile_pages = [&](TileWalker& w, int& p0, int& p1, int& o) {
+      // pages of this thread's tokens in every half of the next tile of walker w (-1 past the end)
+      auto tile_pages = [&](TileWalker& w, int (&p)[H]) {
         int bb, tt, LL;
-        p0 = p1 = -1;
-        o = row_in_half & 63;
+#pragma unroll
+        for (int h = 0; h < H; ++h) p[h] = -1;
         if (!w.next(bb, tt, LL)) return;
         if (a.k_scale == nullptr) return;
-        const int tk0 = tt * kTileTok + row_in_half;
-        if (tk0 < LL) p0 = checked_page(a.block_table, bb, tk0 >> 6, a.max_pages, a.num_pages, a.err);
-        if (tk0 + 128 < LL) p1 = checked_page(a.block_table, bb, (tk0 + 128) >> 6, a.max_pages, a.num_pages, a.err);
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          const int tk = tt * kTileTok + h * 128 + row_in_half;
+          if (tk < LL) p[h] = checked_page(a.block_table, bb, tk >> 6, a.max_pages, a.num_pages, a.err);
+        }
       };
-      auto load_scale = [&](int page, int o) {
-        return page >= 0 ? __ldg(a.k_scale + static_cast<int64_t>(page) * kPage + o) : 1.0f;
+      auto load_scale = [&](int page) {
+        return page >= 0 ? __ldg(a.k_scale + static_cast<int64_t>(page) * kPage + off) : 1.0f;
       };
-      int pa0, pa1, pb0, pb1, pc0, pc1, pd0, pd1, off;
-      tile_pages(w2, pa0, pa1, off);
-      tile_pages(w2, pb0, pb1, off);
-      float ks00 = load_scale(pa0, off), ks01 = load_scale(pa1, off);   // tile +0
-      float ks10 = load_scale(pb0, off), ks11 = load_scale(pb1, off);   // tile +1
+      int pa[H], pb[H], pc[H], pd[H];
+      float ks0[H], ks1[H];
+      tile_pages(w2, pa);
+      tile_pages(w2, pb);
+#pragma unroll
+      for (int h = 0; h < H; ++h) {
+        ks0[h] = load_scale(pa[h]);   // tile +0
+        ks1[h] = load_scale(pb[h]);   // tile +1
+      }
       w4 = w2;
-      tile_pages(w4, pc0, pc1, off);                                    // tile +2
-      tile_pages(w4, pd0, pd1, off);                                    // tile +3
+      tile_pages(w4, pc);             // tile +2
+      tile_pages(w4, pd);             // tile +3
       int b, t, L;
       while (ok && walk.next(b, t, L)) {
-        const float kscale[2] = {ks00, ks01};
-        ks00 = ks10; ks01 = ks11;
-        ks10 = load_scale(pc0, off); ks11 = load_scale(pc1, off);
-        pc0 = pd0; pc1 = pd1;
-        tile_pages(w4, pd0, pd1, off);
+        float kscale[H];
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          kscale[h] = ks0[h];
+          ks0[h] = ks1[h];
+          ks1[h] = load_scale(pc[h]);
+          pc[h] = pd[h];
+        }
+        tile_pages(w4, pd);
         const int tok0 = t * kTileTok;
         for (int g = 0; g < ngroups && ok; ++g) {
-          if (!group_active(a, b, g, tok0, L)) continue;
-          const int q0 = b * a.n_q + g * kQGroup;
-          const int nqg = min(kQGroup, a.n_q - g * kQGroup);
-          for (int h2 = 0; h2 < 2; ++h2, ++unit) {
+          if (!group_active<QG>(a, b, g, tok0, L)) continue;
+          const int q0 = b * a.n_q + g * QG;
+          const int nqg = min(QG, a.n_q - g * QG);
+#pragma unroll
+          for (int u = 0; u < kUnitsPerTile; ++u, ++unit) {
             if ((unit & 1) != eg) continue;
             if (q0 != cur_q0) {
               wb ^= 1;
@@ -371,7 +412,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               for (int i = lane; i < nqg * kHeads; i += 32) {
                 float w = a.head_w[static_cast<int64_t>(q0) * kHeads + i];
                 if (a.q_scale != nullptr) w *= a.q_scale[static_cast<int64_t>(q0) * kHeads + i];
-                wmine[wb * 256 + i] = w;
+                wmine[wb * C::kWPer + i] = w;
               }
               __syncwarp();
               cur_q0 = q0;
@@ -379,27 +420,31 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             const int ab = unit % n_acc;
             if (!wait_warp(&acc_full[ab], (unit / n_acc) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const int tok = tok0 + h2 * 128 + row_in_half;
-            for (int j = 0; j < nqg; ++j) {
-              float acc[64];
-              tmem_ld64(lane_addr + static_cast<uint32_t>(ab * acc_cols + j * kHeads), acc);
-              const float4* wq = reinterpret_cast<const float4*>(wmine + wb * 256 + j * kHeads);
-              float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent chains
 #pragma unroll
-              for (int h4 = 0; h4 < 16; ++h4) {
-                const float4 w = wq[h4];
-                float* pp = part + 4 * (h4 & 1);
-                pp[0] = fmaf(w.x, fmaxf(acc[4 * h4 + 0], 0.0f), pp[0]);
-                pp[1] = fmaf(w.y, fmaxf(acc[4 * h4 + 1], 0.0f), pp[1]);
-                pp[2] = fmaf(w.z, fmaxf(acc[4 * h4 + 2], 0.0f), pp[2]);
-                pp[3] = fmaf(w.w, fmaxf(acc[4 * h4 + 3], 0.0f), pp[3]);
+            for (int hh = 0; hh < UH; ++hh) {
+              const int h2 = u * UH + hh;
+              const int tok = tok0 + h2 * 128 + row_in_half;
+              for (int j = 0; j < nqg; ++j) {
+                float acc[64];
+                tmem_ld64(lane_addr + static_cast<uint32_t>(ab * unit_cols + hh * acc_cols + j * kHeads), acc);
+                const float4* wq = reinterpret_cast<const float4*>(wmine + wb * C::kWPer + j * kHeads);
+                float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent chains
+#pragma unroll
+                for (int h4 = 0; h4 < 16; ++h4) {
+                  const float4 w = wq[h4];
+                  float* pp = part + 4 * (h4 & 1);
+                  pp[0] = fmaf(w.x, fmaxf(acc[4 * h4 + 0], 0.0f), pp[0]);
+                  pp[1] = fmaf(w.y, fmaxf(acc[4 * h4 + 1], 0.0f), pp[1]);
+                  pp[2] = fmaf(w.z, fmaxf(acc[4 * h4 + 2], 0.0f), pp[2]);
+                  pp[3] = fmaf(w.w, fmaxf(acc[4 * h4 + 3], 0.0f), pp[3]);
+                }
+                const float sc =
+                    ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+                const int q = q0 + j;
+                int vis = query_vis(a.q_pos, q, L);
+                if (vis > a.L_max) vis = static_cast<int>(a.L_max);
+                if (tok < vis) a.scores[static_cast<int64_t>(q) * a.L_max + tok] = sc * kscale[h2];
               }
-              const float sc =
-                  ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-              const int q = q0 + j;
-              int vis = query_vis(a.q_pos, q, L);
-              if (vis > a.L_max) vis = static_cast<int>(a.L_max);
-              if (tok < vis) a.scores[static_cast<int64_t>(q) * a.L_max + tok] = sc * kscale[h2];
             }
             tc_fence_before();
             __syncwarp();
@@ -423,7 +468,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
 // Tile prefix over rows (single CTA) plus validation of lengths and causal positions.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q,
-                                                    int max_pages, int32_t* tile_prefix, unsigned int* err) {
+                                                    int max_pages, int tile_tok, int32_t* tile_prefix,
+                                                    unsigned int* err) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
   const int tid = threadIdx.x;
@@ -438,7 +484,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, con
     if (b < B) {
       const int raw = seq_lens[b];
       if (raw < 0 || raw > max_pages * kPage) record_error(err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(raw));
-      tiles = (row_len(seq_lens, b, max_pages) + kTileTok - 1) / kTileTok;
+      tiles = (row_len(seq_lens, b, max_pages) + tile_tok - 1) / tile_tok;
     }
     int v = tiles;
 #pragma unroll
@@ -470,28 +516,36 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, con
 
 
 
-cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages,
+int indexer_tile_tokens(bool fp8, int n_q) {
+  if (n_q == 1) return fp8 ? IdxCfg<1, 1>::kTileTok : IdxCfg<2, 1>::kTileTok;
+  return fp8 ? IdxCfg<1, 4>::kTileTok : IdxCfg<2, 4>::kTileTok;
+}
+
+cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages, int tile_tok,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches) {
-  plan_kernel<<<1, 1024, 0, stream>>>(seq_lens, q_pos, B, n_q, max_pages, tile_prefix, err);
+  plan_kernel<<<1, 1024, 0, stream>>>(seq_lens, q_pos, B, n_q, max_pages, tile_tok, tile_prefix, err);
   ++*launches;
   return cudaGetLastError();
 }
 
-template <int KC>
+template <int KC, int QG>
 static cudaError_t launch_indexer_kc(const CUtensorMap& tk, const CUtensorMap& tq, const IndexerArgs& a, int grid,
                                      cudaStream_t stream) {
-  constexpr int smem = IdxCfg<KC>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  constexpr int smem = IdxCfg<KC, QG>::kSmem;
+  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<KC, QG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  indexer_kernel<KC><<<grid, kIdxThreads, smem, stream>>>(tk, tq, a);
+  indexer_kernel<KC, QG><<<grid, kIdxThreads, smem, stream>>>(tk, tq, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,
                            int grid, cudaStream_t stream, int* launches) {
   ++*launches;
-  return fp8 ? launch_indexer_kc<1>(tmap_k, tmap_q, a, grid, stream)
-             : launch_indexer_kc<2>(tmap_k, tmap_q, a, grid, stream);
+  if (a.n_q == 1)
+    return fp8 ? launch_indexer_kc<1, 1>(tmap_k, tmap_q, a, grid, stream)
+               : launch_indexer_kc<2, 1>(tmap_k, tmap_q, a, grid, stream);
+  return fp8 ? launch_indexer_kc<1, 4>(tmap_k, tmap_q, a, grid, stream)
+             : launch_indexer_kc<2, 4>(tmap_k, tmap_q, a, grid, stream);
 }
 
 }  // namespace dsa

@@ -17,7 +17,7 @@ struct IndexerArgs {
   const float* k_scale;
   float* scores;
   int64_t L_max;
-  const int32_t* tile_prefix;  // [B+1] exclusive prefix of ceil(len/128)
+  const int32_t* tile_prefix;  // [B+1] exclusive prefix of ceil(len / tile tokens)
   unsigned int* err;
 };
 
@@ -56,7 +56,9 @@ struct MlaArgs {
 
 // Each returns the launch error (cudaSuccess when queued) and adds the number of
 // kernels it queued to *launches.
-cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages,
+// Tokens per indexer tile for this cache type and query count (the plan's tile unit).
+int indexer_tile_tokens(bool fp8, int n_q);
+cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages, int tile_tok,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches);
 cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,
                            int grid, cudaStream_t stream, int* launches);
