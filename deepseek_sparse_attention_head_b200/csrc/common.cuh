@@ -110,6 +110,14 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Programmatic dependent launch. Each kernel of the step lets the next one launch early
+// (pdl_trigger) so its CTAs can do their set-up while this kernel finishes; before reading
+// anything a previous kernel of the stream wrote, a kernel waits for the earlier grids to
+// complete and their writes to be visible (pdl_wait). Without the launch attribute both
+// are no-ops.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // One lane of a converged warp (the lowest active one) returns true. tcgen05.mma and
 // tcgen05.commit are issued from such an elected lane of a converged warp: issuing them
 // from a lone divergent thread costs several times more per instruction.

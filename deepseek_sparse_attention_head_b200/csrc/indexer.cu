@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_trigger();
+  pdl_wait();   // the tile prefix comes from the plan kernel
 
   const int total = a.tile_prefix[a.B];
   const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
@@ -473,6 +475,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, con
   __shared__ int warp_sums[32];
   __shared__ int carry;
   const int tid = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (tid == 0) {
     carry = 0;
     tile_prefix[0] = 0;
@@ -523,9 +527,9 @@ int indexer_tile_tokens(bool fp8, int n_q) {
 
 cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages, int tile_tok,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches) {
-  plan_kernel<<<1, 1024, 0, stream>>>(seq_lens, q_pos, B, n_q, max_pages, tile_tok, tile_prefix, err);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, stream, seq_lens, q_pos, B, n_q, max_pages, tile_tok,
+                    tile_prefix, err);
 }
 
 template <int KC, int QG>
@@ -534,8 +538,7 @@ static cudaError_t launch_indexer_kc(const CUtensorMap& tk, const CUtensorMap& t
   constexpr int smem = IdxCfg<KC, QG>::kSmem;
   cudaError_t e = cudaFuncSetAttribute(indexer_kernel<KC, QG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  indexer_kernel<KC, QG><<<grid, kIdxThreads, smem, stream>>>(tk, tq, a);
-  return cudaGetLastError();
+  return launch_pdl(indexer_kernel<KC, QG>, dim3(grid), dim3(kIdxThreads), smem, stream, tk, tq, a);
 }
 
 cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,

@@ -1,6 +1,7 @@
 // Argument blocks and host launchers of the sm_100a kernels (one translation unit per stage).
 #pragma once
 
+#include <utility>
 #include "common.cuh"
 
 namespace dsa {
@@ -53,6 +54,24 @@ struct MlaArgs {
   float* part_o;        // [Bq, nsplit, 64, 512]
   unsigned int* err;
 };
+
+// Launches `kernel` on `stream` with programmatic stream serialisation, so that it may
+// start while the previous kernel in the stream is still running (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Each returns the launch error (cudaSuccess when queued) and adds the number of
 // kernels it queued to *launches.

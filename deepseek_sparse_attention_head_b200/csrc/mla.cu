@@ -198,6 +198,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
   }
 
+  pdl_trigger();
+  pdl_wait();   // the slot list comes from top-k
+
   // the split's slot list, staged once when it fits (invalid entries become -1)
   const bool list_in_smem = ntiles * kMlaTile <= kIdxListCap;
   if (list_in_smem) {
@@ -680,6 +683,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 // Log-sum-exp merge of the split partials: M = max_s m_s, a_s = 2^(m_s - M),
 // out = sum_s a_s o_s / sum_s a_s l_s, lse = (M + log2 sum_s a_s l_s) * ln 2.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+  pdl_trigger();
+  pdl_wait();   // the partials come from the decode kernel
   const int q = blockIdx.x;
   const int h = blockIdx.y;
   const int S = a.nsplit;
@@ -713,17 +718,15 @@ template <bool FP8>
 static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
   if (e != cudaSuccess) return e;
-  mla_decode_kernel<FP8><<<a.Bq * a.nsplit, kMlaThreads, kMlaSmem, stream>>>(tq, a);
-  return cudaGetLastError();
+  return launch_pdl(mla_decode_kernel<FP8>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
 }
 
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
   cudaError_t e = fp8 ? launch_mla_t<true>(tmap_q, a, stream) : launch_mla_t<false>(tmap_q, a, stream);
   ++*launches;
   if (e != cudaSuccess || a.nsplit == 1) return e;
-  mla_combine_kernel<<<dim3(a.Bq, kHeads), 128, 0, stream>>>(a);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(mla_combine_kernel, dim3(a.Bq, kHeads), dim3(128), 0, stream, a);
 }
 
 int mla_tile_keys() { return kMlaTile; }

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
   extern __shared__ uint8_t topk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
 
+  pdl_trigger();
+  pdl_wait();   // scores come from the indexer
   const int tid = threadIdx.x;
   const int q = blockIdx.x;
   const int b = q / a.n_q;
@@ -411,6 +413,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
 // The page-mapping transform alone: physical = table[b, i/64]*64 + i%64, -1 -> -1.
 __global__ void pagemap_kernel(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
                                int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err) {
+  pdl_trigger();
+  pdl_wait();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int q = static_cast<int>(i / top_k);
@@ -435,9 +439,8 @@ cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* lau
   const int smem = static_cast<int>(sizeof(TopkSmem));
   cudaError_t e = cudaFuncSetAttribute(topk_pagemap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  topk_pagemap_kernel<<<Bq, kTopkThreads, smem, stream>>>(a);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(topk_pagemap_kernel, dim3(Bq), dim3(kTopkThreads), smem, stream, a);
 }
 
 cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
@@ -446,10 +449,9 @@ cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* blo
   int64_t blocks = (total + 255) / 256;
   if (blocks > 4096) blocks = 4096;
   if (blocks < 1) blocks = 1;
-  pagemap_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(n_q, top_k, total, block_table, max_pages, num_pages,
-                                                               logical, physical, err);
   ++*launches;
-  return cudaGetLastError();
+  return launch_pdl(pagemap_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, n_q, top_k, total,
+                    block_table, max_pages, num_pages, logical, physical, err);
 }
 
 }  // namespace dsa
