@@ -90,6 +90,9 @@ int mla_splits_for(int Bq, int top_k, int* keys_per_split) {
 
 struct Layout {
   size_t prefix = 0, scores = 0, logical = 0, physical = 0, part_ml = 0, part_o = 0, total = 0;
+  // long-row top-k: per-query count / max / threshold words and candidate buffers
+  int tk_chunks = 1;
+  size_t tk_meta = 0, tk_key = 0, tk_idx = 0;
 };
 
 // op: DSA_OP_* or -1 for the MLA call alone.
@@ -107,6 +110,19 @@ Layout layout_for(int B, int64_t Bq, int64_t L_max, int top_k, int op, int nspli
     off += up256(static_cast<size_t>(Bq) * top_k * 4);
     l.physical = off;
     off += up256(static_cast<size_t>(Bq) * top_k * 4);
+  }
+  if (op == DSA_OP_TOPK || op == DSA_OP_LAYER) {
+    const int ch = topk_chunks(static_cast<int>(Bq), L_max, device_sms());
+    if (ch > 1) {
+      const size_t cap = static_cast<size_t>(topk_candidate_capacity());
+      l.tk_chunks = ch;
+      l.tk_meta = off;
+      off += up256(static_cast<size_t>(Bq) * 3 * 4);
+      l.tk_key = off;
+      off += up256(static_cast<size_t>(Bq) * cap * 4);
+      l.tk_idx = off;
+      off += up256(static_cast<size_t>(Bq) * cap * 4);
+    }
   }
   if ((op == DSA_OP_LAYER || op == -1) && nsplit > 1) {
     l.part_ml = off;
@@ -161,8 +177,16 @@ dsa_status run_indexer(const dsa_paging* pg, const void* q_idx, dsa_dtype dt, co
   return cuda_status(launch_indexer(fp8, tk, tq, a, grid, st, &g_launches));
 }
 
+// Zeroes the long-row top-k counters (count, max, threshold per query) of a layout.
+dsa_status clear_topk_counters(const Layout& lay, int64_t Bq, uint8_t* ws, cudaStream_t st) {
+  if (lay.tk_chunks <= 1) return DSA_OK;
+  return cuda_status(cudaMemsetAsync(ws + lay.tk_meta, 0, static_cast<size_t>(Bq) * 3 * 4, st));
+}
+
+// `counters_clear`: the long-row counters were zeroed earlier on this stream.
 dsa_status run_topk(const dsa_paging* pg, const float* scores, int64_t L_max, int top_k, int32_t* logical,
-                    int32_t* physical, uint8_t* ws, cudaStream_t st) {
+                    int32_t* physical, uint8_t* ws, const Layout& lay, bool counters_clear, cudaStream_t st) {
+  const int64_t Bq = static_cast<int64_t>(pg->B) * pg->n_q;
   TopkArgs a;
   a.n_q = pg->n_q;
   a.seq_lens = pg->seq_lens;
@@ -176,7 +200,23 @@ dsa_status run_topk(const dsa_paging* pg, const float* scores, int64_t L_max, in
   a.logical = logical;
   a.physical = physical;
   a.err = err_word(ws);
-  return cuda_status(launch_topk(a, pg->B * pg->n_q, st, &g_launches));
+  a.chunks = lay.tk_chunks;
+  a.cand_cap = topk_candidate_capacity();
+  a.g_cnt = a.g_rmax = a.g_thr = a.g_key = nullptr;
+  a.g_idx = nullptr;
+  if (lay.tk_chunks > 1) {
+    uint32_t* meta = reinterpret_cast<uint32_t*>(ws + lay.tk_meta);
+    a.g_cnt = meta;
+    a.g_rmax = meta + Bq;
+    a.g_thr = meta + 2 * Bq;
+    a.g_key = reinterpret_cast<uint32_t*>(ws + lay.tk_key);
+    a.g_idx = reinterpret_cast<int32_t*>(ws + lay.tk_idx);
+    if (!counters_clear) {
+      const dsa_status s = clear_topk_counters(lay, Bq, ws, st);
+      if (s != DSA_OK) return s;
+    }
+  }
+  return cuda_status(launch_topk(a, static_cast<int>(Bq), st, &g_launches));
 }
 
 dsa_status run_mla(int Bq, const void* q, const void* kv, dsa_dtype kv_dtype, const float* kv_scale,
@@ -299,10 +339,12 @@ dsa_status dsa_topk_pagemap(const dsa_paging* paging, const float* scores, int64
   if (s != DSA_OK) return s;
   if (scores == nullptr || L_max < 1 || top_k < 1 || top_k > 16384) return DSA_ERR_INVALID_ARG;
   if (logical_out == nullptr && physical_out == nullptr) return DSA_ERR_INVALID_ARG;
-  s = check_ws(workspace, ws_bytes, layout_for(paging->B, 0, L_max, top_k, DSA_OP_TOPK, 1).total);
+  const int64_t Bq = static_cast<int64_t>(paging->B) * paging->n_q;
+  const Layout lay = layout_for(paging->B, Bq, L_max, top_k, DSA_OP_TOPK, 1);
+  s = check_ws(workspace, ws_bytes, lay.total);
   if (s != DSA_OK) return s;
-  return run_topk(paging, scores, L_max, top_k, logical_out, physical_out, static_cast<uint8_t*>(workspace),
-                  static_cast<cudaStream_t>(stream));
+  return run_topk(paging, scores, L_max, top_k, logical_out, physical_out, static_cast<uint8_t*>(workspace), lay,
+                  false, static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_pagemap(const dsa_paging* paging, const int32_t* logical, int32_t top_k, int32_t* physical,
@@ -362,9 +404,12 @@ dsa_status dsa_decode_layer(const dsa_paging* paging, const void* q_idx, dsa_dty
   float* scores = reinterpret_cast<float*>(ws + lay.scores);
   int32_t* logical = logical_out ? logical_out : reinterpret_cast<int32_t*>(ws + lay.logical);
   int32_t* physical = physical_out ? physical_out : reinterpret_cast<int32_t*>(ws + lay.physical);
+  // cleared here, ahead of the first kernel, so the top-k follows the indexer directly
+  s = clear_topk_counters(lay, Bq, ws, st);
+  if (s != DSA_OK) return s;
   s = run_indexer(paging, q_idx, idx_dtype, q_scale, head_w, k_cache, k_scale, scores, L_layer, ws, lay, st);
   if (s != DSA_OK) return s;
-  s = run_topk(paging, scores, L_layer, top_k, logical, physical, ws, st);
+  s = run_topk(paging, scores, L_layer, top_k, logical, physical, ws, lay, true, st);
   if (s != DSA_OK) return s;
   return run_mla(static_cast<int>(Bq), q_mla, kv_cache, kv_dtype, kv_scale, num_slots, physical, top_k,
                  softmax_scale, out, out_dtype, lse, ws, lay, nsplit, kps, st);

@@ -536,7 +536,7 @@ template <int KC, int QG>
 static cudaError_t launch_indexer_kc(const CUtensorMap& tk, const CUtensorMap& tq, const IndexerArgs& a, int grid,
                                      cudaStream_t stream) {
   constexpr int smem = IdxCfg<KC, QG>::kSmem;
-  cudaError_t e = cudaFuncSetAttribute(indexer_kernel<KC, QG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_smem_once<indexer_kernel<KC, QG>>(smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(indexer_kernel<KC, QG>, dim3(grid), dim3(kIdxThreads), smem, stream, tk, tq, a);
 }

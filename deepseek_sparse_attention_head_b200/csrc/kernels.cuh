@@ -1,6 +1,7 @@
 // Argument blocks and host launchers of the sm_100a kernels (one translation unit per stage).
 #pragma once
 
+#include <atomic>
 #include <utility>
 #include "common.cuh"
 
@@ -35,6 +36,15 @@ struct TopkArgs {
   int32_t* logical;   // may be null
   int32_t* physical;  // may be null
   unsigned int* err;
+  // long-row gather (chunks > 1): per-query candidate count, largest key - threshold,
+  // threshold, and candidate buffers [Bq, cand_cap]; counts and maxima start at zero
+  int chunks;
+  int cand_cap;
+  uint32_t* g_cnt;
+  uint32_t* g_rmax;
+  uint32_t* g_thr;
+  uint32_t* g_key;
+  int32_t* g_idx;
 };
 
 struct MlaArgs {
@@ -54,6 +64,21 @@ struct MlaArgs {
   float* part_o;        // [Bq, nsplit, 64, 512]
   unsigned int* err;
 };
+
+// Raises kernel K's dynamic shared-memory limit once per device (a host-side cost that
+// would otherwise be paid on every launch). One flag word per kernel.
+template <auto K>
+inline cudaError_t set_smem_once(int bytes) {
+  static std::atomic<uint64_t> done{0};   // one bit per device ordinal < 64
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launches `kernel` on `stream` with programmatic stream serialisation, so that it may
 // start while the previous kernel in the stream is still running (see pdl_wait).
@@ -81,6 +106,9 @@ cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, in
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches);
 cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,
                            int grid, cudaStream_t stream, int* launches);
+// Chunks per row of the long-row top-k (1 = one CTA per query) and its candidate capacity.
+int topk_chunks(int Bq, int64_t L_max, int sms);
+int topk_candidate_capacity();
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches);
 cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
                            int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,

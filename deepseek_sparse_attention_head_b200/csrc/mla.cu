@@ -716,7 +716,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
 
 template <bool FP8>
 static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
+  cudaError_t e = set_smem_once<mla_decode_kernel<FP8>>(kMlaSmem);
   if (e != cudaSuccess) return e;
   return launch_pdl(mla_decode_kernel<FP8>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
 }

@@ -3,8 +3,9 @@
 // usage: SGLANG_NSA_FUSE_TOPK=1 fuses the page-mapping transform into top-k).
 //
 // One CTA per query. Scores are mapped to order-preserving 32-bit keys.
-//  1. A threshold is estimated from 256 evenly spaced samples of the row, low enough
-//     that about 1.25 k / vis of the samples (plus a margin) lie above it.
+//  1. A threshold is estimated from evenly spaced samples of the row (256, or up to
+//     4096 for very long rows), low enough that about 1.25 k / vis of the samples (plus
+//     a margin) lie above it.
 //  2. One pass over the row gathers every key at or above the threshold into shared
 //     memory (per-thread counts, a warp prefix sum and one shared atomic per warp for
 //     every 16K keys).
@@ -13,6 +14,9 @@
 //     histograms), and the winners are emitted with their physical slots.
 // When the estimate misses (fewer than k candidates, or more than fit), a
 // three-digit radix select over the whole row (12 + 12 + 8 bits) decides instead.
+// Few very long rows (the 1M-token stream) split step 2 over 16K-key
+// chunks, one CTA each, into a per-row candidate buffer in the workspace; a second
+// kernel then runs step 3 per row.
 // A query that sees no more than top_k tokens takes all of them (the dense path).
 #include "kernels.cuh"
 
@@ -27,6 +31,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 constexpr int kTopkThreads = 1024;
 constexpr int kHistBins = 4096;
 constexpr int kCand = 12288;  // candidates kept in shared memory
+constexpr int kTopkChunk = 16384;   // keys per CTA of the long-row gather
 
 struct TopkSmem {
   uint32_t hist[kHistBins];
@@ -128,57 +133,89 @@ __device__ __forceinline__ uint32_t warp_reserve(uint32_t* counter, uint32_t n) 
   return base + incl - n;
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkArgs a) {
-  extern __shared__ uint8_t topk_smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+// Per-row context shared by the phases below.
+struct TopkRow {
+  int q, b, vis, K;
+  const float* row;
+  int32_t* lo;   // logical out row, or null
+  int32_t* po;   // physical out row, or null
+};
 
-  pdl_trigger();
-  pdl_wait();   // scores come from the indexer
-  const int tid = threadIdx.x;
-  const int q = blockIdx.x;
-  const int b = q / a.n_q;
-  const int L = row_len(a.seq_lens, b, a.max_pages);
-  int vis = query_vis(a.q_pos, q, L);
-  if (vis > a.L_max) vis = static_cast<int>(a.L_max);
-  const int K = a.top_k;
-  int32_t* lo = a.logical ? a.logical + static_cast<int64_t>(q) * K : nullptr;
-  int32_t* po = a.physical ? a.physical + static_cast<int64_t>(q) * K : nullptr;
+__device__ __forceinline__ TopkRow topk_row(const TopkArgs& a, int q) {
+  TopkRow r;
+  r.q = q;
+  r.b = q / a.n_q;
+  const int L = row_len(a.seq_lens, r.b, a.max_pages);
+  r.vis = query_vis(a.q_pos, q, L);
+  if (r.vis > a.L_max) r.vis = static_cast<int>(a.L_max);
+  r.K = a.top_k;
+  r.row = a.scores + static_cast<int64_t>(q) * a.L_max;
+  r.lo = a.logical ? a.logical + static_cast<int64_t>(q) * r.K : nullptr;
+  r.po = a.physical ? a.physical + static_cast<int64_t>(q) * r.K : nullptr;
+  return r;
+}
 
-  auto emit = [&](int pos, int s) {
-    if (lo) lo[pos] = s;
-    if (po) {
-      int slot = -1;
-      if (s >= 0) slot = checked_page(a.block_table, b, s >> 6, a.max_pages, a.num_pages, a.err) * kPage + (s & 63);
-      po[pos] = slot;
-    }
-  };
-
-  if (vis <= K) {  // dense path: every visible token
-    for (int i = tid; i < K; i += kTopkThreads) emit(i, i < vis ? i : -1);
-    return;
+__device__ __forceinline__ void topk_emit(const TopkArgs& a, const TopkRow& r, int pos, int s) {
+  if (r.lo) r.lo[pos] = s;
+  if (r.po) {
+    int slot = -1;
+    if (s >= 0) slot = checked_page(a.block_table, r.b, s >> 6, a.max_pages, a.num_pages, a.err) * kPage + (s & 63);
+    r.po[pos] = slot;
   }
+}
 
-  const float* row = a.scores + static_cast<int64_t>(q) * a.L_max;
+// Dense path: every visible token (vis <= top_k).
+__device__ __forceinline__ void topk_dense(const TopkArgs& a, const TopkRow& r) {
+  for (int i = threadIdx.x; i < r.K; i += kTopkThreads) topk_emit(a, r, i, i < r.vis ? i : -1);
+}
 
-  // The sampled path needs 16-byte aligned rows (always true for the fused layer, whose
-  // row stride is a multiple of 64); other rows take the whole-row radix select below.
-  const bool aligned_row = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
-  if (aligned_row) {
-  // ---- 1. threshold from 256 evenly spaced samples (kept in the histogram area)
+// Threshold estimate (whole CTA): S = min(4096, vis) evenly spaced samples of the row, and
+// a key at or below the `need`-th largest sample, need = 1.25 E + 3 sqrt(E) + 4 with
+// E = S k / vis the expected number of true top-k keys among the samples. Found by a
+// two-digit histogram select (bits 31..20, then 19..8) and rounded down to its 24-bit
+// prefix. Deterministic: every CTA that calls it on the same row gets the same value.
+// Uses sm.hist and sm.cand_key[0..S).
+__device__ uint32_t row_threshold(TopkSmem& sm, const float* row, int vis, int K) {
+  constexpr int kMaxSamples = 4096;
+  const int tid = threadIdx.x;
+  const int S = min(kMaxSamples, vis);
+  for (int i = tid; i < S; i += kTopkThreads)
+    sm.cand_key[i] = order_key(__ldg(row + static_cast<int>((static_cast<int64_t>(i) * vis) / S)));
+  const float expect = static_cast<float>(S) * static_cast<float>(K) / static_cast<float>(vis);
+  const uint32_t need = static_cast<uint32_t>(
+      fminf(1.25f * expect + 3.0f * sqrtf(expect) + 4.0f, static_cast<float>(S)));
+  for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < S; i += kTopkThreads) atomicAdd(&sm.hist[sm.cand_key[i] >> 20], 1u);
+  __syncthreads();
+  select_bin(sm, need);
+  const uint32_t b1 = sm.sel_bin, r1 = sm.sel_rem;
+  for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < S; i += kTopkThreads) {
+    const uint32_t u = sm.cand_key[i];
+    if ((u >> 20) == b1) atomicAdd(&sm.hist[(u >> 8) & 0xFFFu], 1u);
+  }
+  __syncthreads();
+  select_bin(sm, r1);
+  const uint32_t thr = (b1 << 20) | (sm.sel_bin << 8);
+  __syncthreads();   // sm.cand_key is reused by the caller
+  return thr;
+}
+
+// Threshold estimate for one CTA per row: 256 evenly spaced samples, each ranked against
+// all the others; the largest sample with at least need = 1.25 E + 3 sqrt(E) + 4 samples
+// above it (E = 256 k / vis). Cheaper than row_threshold for rows of up to ~64K keys.
+__device__ uint32_t row_threshold_small(TopkSmem& sm, const float* row, int vis, int K) {
   constexpr int kSamples = 256;
+  const int tid = threadIdx.x;
   uint32_t* samp = sm.hist;
   uint32_t mykey = 0u;
   if (tid < kSamples) {
-    mykey = order_key(row[static_cast<int>((static_cast<int64_t>(tid) * vis) / kSamples)]);
+    mykey = order_key(__ldg(row + static_cast<int>((static_cast<int64_t>(tid) * vis) / kSamples)));
     samp[tid] = mykey;
   }
-  if (tid == 0) {
-    sm.thr = 0u;
-    sm.rmax = 0u;
-    sm.n_cand = 0;
-    sm.cnt_out = 0;
-    sm.cnt_eq = 0;
-  }
+  if (tid == 0) sm.thr = 0u;
   __syncthreads();
   if (tid < kSamples) {
     uint32_t above = 0;      // samples strictly above this thread's sample
@@ -190,147 +227,164 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
     }
     const float expect = static_cast<float>(kSamples) * static_cast<float>(K) / static_cast<float>(vis);
     const uint32_t need = static_cast<uint32_t>(fminf(1.25f * expect + 3.0f * sqrtf(expect) + 4.0f, 1e9f));
-    // the largest sample with at least `need` samples above it
     const uint32_t cand = above >= need ? mykey : 0u;
     const uint32_t wmax = __reduce_max_sync(0xffffffffu, cand);
     if ((tid & 31) == 0 && wmax != 0u) atomicMax(&sm.thr, wmax);
   }
   __syncthreads();
   const uint32_t thr = sm.thr;
+  __syncthreads();   // sm.hist is reused by the caller
+  return thr;
+}
 
-  // ---- 2. gather every key >= thr (coalesced, convergent; ballot compaction)
-  {
-    // Batches of 16 keys per thread (four 16-byte loads, coalesced across the block); the
-    // next batch is loaded before this one is processed. One slot reservation per warp and
-    // batch. The row start is 16-byte aligned (the row stride is a multiple of 64 floats).
-    constexpr int kU = 16;
-    constexpr int kBatch = kU * kTopkThreads;
-    const float4* r4 = reinterpret_cast<const float4*>(row);
-    auto load_batch = [&](int base, float4 (&v)[kU / 4]) {
+// Gathers every key >= thr of row[lo_s, hi_s) (lo_s a multiple of 4, the row 16-byte
+// aligned) into out_key / out_idx at slots reserved from *counter (shared or global; one
+// atomic per warp per 16K keys; slots >= cap are counted but not stored), and raises
+// *rmax_addr to the largest key - thr. Whole CTA; the trip count is CTA-uniform.
+__device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr, uint32_t* counter,
+                             uint32_t* out_key, int32_t* out_idx, uint32_t cap, uint32_t* rmax_addr) {
+  constexpr int kU = 16;
+  constexpr int kBatch = kU * kTopkThreads;
+  const int tid = threadIdx.x;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  auto load_batch = [&](int base, float4 (&v)[kU / 4]) {
 #pragma unroll
-      for (int j = 0; j < kU / 4; ++j) {
-        const int s_ = base + 4 * (j * kTopkThreads + tid);
-        v[j] = s_ + 3 < vis ? __ldg(r4 + (s_ >> 2))
-                            : make_float4(s_ < vis ? row[s_] : 0.0f, s_ + 1 < vis ? row[s_ + 1] : 0.0f,
-                                          s_ + 2 < vis ? row[s_ + 2] : 0.0f, 0.0f);
-      }
-    };
-    uint32_t lmax = 0;
-    float4 cur[kU / 4], nxt[kU / 4];
-    load_batch(0, cur);
-    for (int base = 0; base < vis; base += kBatch) {
-      if (base + kBatch < vis) load_batch(base + kBatch, nxt);
-      uint32_t takes = 0;
+    for (int j = 0; j < kU / 4; ++j) {
+      const int s_ = base + 4 * (j * kTopkThreads + tid);
+      v[j] = s_ + 3 < hi_s ? __ldg(r4 + (s_ >> 2))
+                           : make_float4(s_ < hi_s ? row[s_] : 0.0f, s_ + 1 < hi_s ? row[s_ + 1] : 0.0f,
+                                         s_ + 2 < hi_s ? row[s_ + 2] : 0.0f, 0.0f);
+    }
+  };
+  uint32_t lmax = 0;
+  float4 cur[kU / 4], nxt[kU / 4];
+  load_batch(lo_s, cur);
+  for (int base = lo_s; base < hi_s; base += kBatch) {
+    if (base + kBatch < hi_s) load_batch(base + kBatch, nxt);
+    uint32_t takes = 0;
 #pragma unroll
-      for (int j = 0; j < kU / 4; ++j) {
-        const int s_ = base + 4 * (j * kTopkThreads + tid);
-        const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+    for (int j = 0; j < kU / 4; ++j) {
+      const int s_ = base + 4 * (j * kTopkThreads + tid);
+      const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
-          if (s_ + t < vis && order_key(e[t]) >= thr) takes |= 1u << (4 * j + t);
-      }
-      uint32_t c = warp_reserve(&sm.n_cand, static_cast<uint32_t>(__popc(takes)));
+      for (int t = 0; t < 4; ++t)
+        if (s_ + t < hi_s && order_key(e[t]) >= thr) takes |= 1u << (4 * j + t);
+    }
+    uint32_t c = warp_reserve(counter, static_cast<uint32_t>(__popc(takes)));
 #pragma unroll
-      for (int j = 0; j < kU / 4; ++j) {
-        const int s_ = base + 4 * (j * kTopkThreads + tid);
-        const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+    for (int j = 0; j < kU / 4; ++j) {
+      const int s_ = base + 4 * (j * kTopkThreads + tid);
+      const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          if (takes & (1u << (4 * j + t))) {
-            const uint32_t u = order_key(e[t]);
-            if (c < static_cast<uint32_t>(kCand)) {
-              sm.cand_key[c] = u;
-              sm.cand_idx[c] = s_ + t;
-            }
-            ++c;
-            lmax = max(lmax, u - thr);
+      for (int t = 0; t < 4; ++t) {
+        if (takes & (1u << (4 * j + t))) {
+          const uint32_t u = order_key(e[t]);
+          if (c < cap) {
+            out_key[c] = u;
+            out_idx[c] = s_ + t;
           }
+          ++c;
+          lmax = max(lmax, u - thr);
         }
       }
-#pragma unroll
-      for (int j = 0; j < kU / 4; ++j) cur[j] = nxt[j];
     }
-    const uint32_t wmax = __reduce_max_sync(0xffffffffu, lmax);
-    if ((tid & 31) == 0) atomicMax(&sm.rmax, wmax);
+#pragma unroll
+    for (int j = 0; j < kU / 4; ++j) cur[j] = nxt[j];
   }
-  __syncthreads();
-  const uint32_t n_c = sm.n_cand;
-  if (n_c >= static_cast<uint32_t>(K) && n_c <= static_cast<uint32_t>(kCand)) {
-    // ---- 3. exact radix select over r = key - thr among the candidates
-    const uint32_t rmax = sm.rmax;
-    int hi = rmax == 0u ? 0 : 32 - __clz(rmax);          // r fits in bits [0, hi)
-    uint32_t prefix = 0u, pmask = 0u, remaining = static_cast<uint32_t>(K);
-#pragma unroll 1
-    while (true) {
-      const int lo_bit = hi > 12 ? hi - 12 : 0;
-      const uint32_t dm = (1u << (hi - lo_bit)) - 1u;      // hi - lo_bit in [0, 12]
-      for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
-      __syncthreads();
-      for (int c = tid; c < static_cast<int>(n_c); c += kTopkThreads) {
-        const uint32_t r = sm.cand_key[c] - thr;
-        if ((r & pmask) == prefix) atomicAdd(&sm.hist[(r >> lo_bit) & dm], 1u);
-      }
-      __syncthreads();
-      select_bin(sm, remaining);
-      prefix |= sm.sel_bin << lo_bit;
-      pmask |= dm << lo_bit;
-      remaining = sm.sel_rem;
-      if (lo_bit == 0) break;
-      hi = lo_bit;
-    }
-    const uint32_t kth = prefix, take_eq = remaining;
-    const uint32_t n_gt = static_cast<uint32_t>(K) - take_eq;
-    // emit: each thread takes candidates tid, tid + 1024, ... (at most kCand / 1024)
-    constexpr int kPer = kCand / kTopkThreads;
-    uint32_t gts = 0, eqs = 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int c = j * kTopkThreads + tid;
-      if (c < static_cast<int>(n_c)) {
-        const uint32_t r = sm.cand_key[c] - thr;
-        if (r > kth) gts |= 1u << j;
-        else if (r == kth) eqs |= 1u << j;
-      }
-    }
-    uint32_t pg = warp_reserve(&sm.cnt_out, static_cast<uint32_t>(__popc(gts)));
-    uint32_t pe = warp_reserve(&sm.cnt_eq, static_cast<uint32_t>(__popc(eqs)));
-    // output positions and tokens first, then all block-table lookups, then the stores
-    int pos[kPer], tok[kPer], page[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      pos[j] = -1;
-      tok[j] = 0;
-      const int c = j * kTopkThreads + tid;
-      if (gts & (1u << j)) {
-        if (pg < n_gt) { pos[j] = static_cast<int>(pg); tok[j] = sm.cand_idx[c]; }
-        ++pg;
-      } else if (eqs & (1u << j)) {
-        if (pe < take_eq) { pos[j] = static_cast<int>(n_gt + pe); tok[j] = sm.cand_idx[c]; }
-        ++pe;
-      }
-    }
-    const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_pages;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) page[j] = (po != nullptr && pos[j] >= 0) ? __ldg(bt_row + (tok[j] >> 6)) : 0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (page[j] < 0 || page[j] >= a.num_pages) {
-        if (pos[j] >= 0) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(page[j]));
-        page[j] = 0;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (pos[j] < 0) continue;
-      if (lo) lo[pos[j]] = tok[j];
-      if (po) po[pos[j]] = page[j] * kPage + (tok[j] & 63);
-    }
-    return;
-  }
-  __syncthreads();
-  }   // aligned_row
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, lmax);
+  if ((tid & 31) == 0 && wmax != 0u) atomicMax(rmax_addr, wmax);
+}
 
-  // ---- fallback: digit 1 (key bits 31..20) over the whole row
+// Exact selection among the n_c shared-memory candidates (all keys >= thr, n_c in
+// [K, kCand]): radix select over r = key - thr in 12-bit digits, then emission of the keys
+// above the k-th and the needed number equal to it. Whole CTA.
+__device__ void select_and_emit(TopkSmem& sm, const TopkArgs& a, const TopkRow& rw, uint32_t n_c, uint32_t thr,
+                                uint32_t rmax) {
+  const int tid = threadIdx.x;
+  const int K = rw.K;
+  if (tid == 0) {
+    sm.cnt_out = 0;
+    sm.cnt_eq = 0;
+  }
+  int hi = rmax == 0u ? 0 : 32 - __clz(rmax);          // r fits in bits [0, hi)
+  uint32_t prefix = 0u, pmask = 0u, remaining = static_cast<uint32_t>(K);
+#pragma unroll 1
+  while (true) {
+    const int lo_bit = hi > 12 ? hi - 12 : 0;
+    const uint32_t dm = (1u << (hi - lo_bit)) - 1u;      // hi - lo_bit in [0, 12]
+    for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (int c = tid; c < static_cast<int>(n_c); c += kTopkThreads) {
+      const uint32_t r = sm.cand_key[c] - thr;
+      if ((r & pmask) == prefix) atomicAdd(&sm.hist[(r >> lo_bit) & dm], 1u);
+    }
+    __syncthreads();
+    select_bin(sm, remaining);
+    prefix |= sm.sel_bin << lo_bit;
+    pmask |= dm << lo_bit;
+    remaining = sm.sel_rem;
+    if (lo_bit == 0) break;
+    hi = lo_bit;
+  }
+  const uint32_t kth = prefix, take_eq = remaining;
+  const uint32_t n_gt = static_cast<uint32_t>(K) - take_eq;
+  // each thread takes candidates tid, tid + 1024, ... (at most kCand / 1024)
+  constexpr int kPer = kCand / kTopkThreads;
+  uint32_t gts = 0, eqs = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int c = j * kTopkThreads + tid;
+    if (c < static_cast<int>(n_c)) {
+      const uint32_t r = sm.cand_key[c] - thr;
+      if (r > kth) gts |= 1u << j;
+      else if (r == kth) eqs |= 1u << j;
+    }
+  }
+  uint32_t pg = warp_reserve(&sm.cnt_out, static_cast<uint32_t>(__popc(gts)));
+  uint32_t pe = warp_reserve(&sm.cnt_eq, static_cast<uint32_t>(__popc(eqs)));
+  // output positions and tokens first, then all block-table lookups, then the stores
+  int pos[kPer], tok[kPer], page[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    pos[j] = -1;
+    tok[j] = 0;
+    const int c = j * kTopkThreads + tid;
+    if (gts & (1u << j)) {
+      if (pg < n_gt) { pos[j] = static_cast<int>(pg); tok[j] = sm.cand_idx[c]; }
+      ++pg;
+    } else if (eqs & (1u << j)) {
+      if (pe < take_eq) { pos[j] = static_cast<int>(n_gt + pe); tok[j] = sm.cand_idx[c]; }
+      ++pe;
+    }
+  }
+  const int32_t* bt_row = a.block_table + static_cast<int64_t>(rw.b) * a.max_pages;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) page[j] = (rw.po != nullptr && pos[j] >= 0) ? __ldg(bt_row + (tok[j] >> 6)) : 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (page[j] < 0 || page[j] >= a.num_pages) {
+      if (pos[j] >= 0) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(page[j]));
+      page[j] = 0;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (pos[j] < 0) continue;
+    if (rw.lo) rw.lo[pos[j]] = tok[j];
+    if (rw.po) rw.po[pos[j]] = page[j] * kPage + (tok[j] & 63);
+  }
+}
+
+// Whole-row exact radix select (12 + 12 + 8 bits); for rows where the sampled path missed
+// or the row is not 16-byte aligned. Whole CTA.
+__device__ void select_whole_row(TopkSmem& sm, const TopkArgs& a, const TopkRow& rw) {
+  const int tid = threadIdx.x;
+  const int K = rw.K;
+  const int vis = rw.vis;
+  const float* row = rw.row;
+  auto emit = [&](int pos, int s) { topk_emit(a, rw, pos, s); };
+  __syncthreads();
+  // digit 1 (key bits 31..20) over the whole row
   for (int i = tid; i < kHistBins; i += kTopkThreads) sm.hist[i] = 0;
   if (tid == 0) {
     sm.n_cand = 0;
@@ -410,6 +464,85 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
   }
 }
 
+// One CTA per query: threshold, gather into shared memory, exact select.
+__global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkArgs a) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  pdl_trigger();
+  pdl_wait();   // scores come from the indexer
+  const TopkRow rw = topk_row(a, blockIdx.x);
+  if (rw.vis <= rw.K) {
+    topk_dense(a, rw);
+    return;
+  }
+  // The sampled path needs 16-byte aligned rows (always true for the fused layer, whose
+  // row stride is a multiple of 64); other rows take the whole-row radix select.
+  if ((reinterpret_cast<uintptr_t>(rw.row) & 15) == 0) {
+    const uint32_t thr = row_threshold_small(sm, rw.row, rw.vis, rw.K);
+    if (threadIdx.x == 0) {
+      sm.n_cand = 0;
+      sm.rmax = 0;
+    }
+    __syncthreads();
+    gather_range(rw.row, 0, rw.vis, thr, &sm.n_cand, sm.cand_key, sm.cand_idx, kCand, &sm.rmax);
+    __syncthreads();
+    const uint32_t n_c = sm.n_cand;
+    if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand)) {
+      select_and_emit(sm, a, rw, n_c, thr, sm.rmax);
+      return;
+    }
+  }
+  select_whole_row(sm, a, rw);
+}
+
+// Long rows, part 1: grid (chunks, queries). Each CTA derives the row's threshold (the same
+// in every chunk CTA) and gathers the candidates of its 16K-key chunk into the row's
+// global candidate buffer.
+__global__ void __launch_bounds__(kTopkThreads) topk_gather_kernel(const TopkArgs a) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  pdl_trigger();
+  pdl_wait();   // scores come from the indexer
+  const TopkRow rw = topk_row(a, blockIdx.y);
+  if (rw.vis <= rw.K || (reinterpret_cast<uintptr_t>(rw.row) & 15) != 0) return;   // handled by part 2
+  const int lo_s = static_cast<int>(blockIdx.x) * kTopkChunk;
+  if (lo_s >= rw.vis) return;
+  const int hi_s = min(rw.vis, lo_s + kTopkChunk);
+  const uint32_t thr = row_threshold(sm, rw.row, rw.vis, rw.K);
+  const int64_t q = rw.q;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.g_thr[q] = thr;
+  gather_range(rw.row, lo_s, hi_s, thr, a.g_cnt + q, a.g_key + q * a.cand_cap, a.g_idx + q * a.cand_cap,
+               static_cast<uint32_t>(a.cand_cap), a.g_rmax + q);
+}
+
+// Long rows, part 2: one CTA per query selects exactly among the gathered candidates
+// (or the whole row when the estimate missed) and emits logical and physical indices.
+__global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const TopkArgs a) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  pdl_trigger();
+  pdl_wait();   // candidates come from part 1
+  const TopkRow rw = topk_row(a, blockIdx.x);
+  if (rw.vis <= rw.K) {
+    topk_dense(a, rw);
+    return;
+  }
+  const int64_t q = rw.q;
+  const uint32_t n_c = a.g_cnt[q];
+  if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand) && n_c <= static_cast<uint32_t>(a.cand_cap)) {
+    const uint32_t* gk = a.g_key + q * a.cand_cap;
+    const int32_t* gi = a.g_idx + q * a.cand_cap;
+    for (int i = threadIdx.x; i < static_cast<int>(n_c); i += kTopkThreads) {
+      sm.cand_key[i] = gk[i];
+      sm.cand_idx[i] = gi[i];
+    }
+    __syncthreads();
+    select_and_emit(sm, a, rw, n_c, a.g_thr[q], a.g_rmax[q]);
+    return;
+  }
+  select_whole_row(sm, a, rw);
+}
+
 // The page-mapping transform alone: physical = table[b, i/64]*64 + i%64, -1 -> -1.
 __global__ void pagemap_kernel(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
                                int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err) {
@@ -435,12 +568,34 @@ __global__ void pagemap_kernel(int n_q, int top_k, int64_t total, const int32_t*
   }
 }
 
+int topk_chunks(int Bq, int64_t L_max, int sms) {
+  // Very long rows (at least 128K keys) and few of them: split the gather over 16K-key
+  // chunks, up to two CTAs per SM. Shorter rows are faster with one CTA each.
+  if (Bq <= 0 || sms <= 0 || Bq >= sms || L_max < 8 * static_cast<int64_t>(kTopkChunk)) return 1;
+  const int64_t want = (L_max + kTopkChunk - 1) / kTopkChunk;
+  const int64_t room = (2 * static_cast<int64_t>(sms)) / Bq;
+  const int64_t c = want < room ? want : room;
+  return c < 2 ? 1 : static_cast<int>(c);
+}
+
+int topk_candidate_capacity() { return kCand; }
+
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches) {
   const int smem = static_cast<int>(sizeof(TopkSmem));
-  cudaError_t e = cudaFuncSetAttribute(topk_pagemap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (a.chunks <= 1) {
+    cudaError_t e = set_smem_once<topk_pagemap_kernel>(smem);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    return launch_pdl(topk_pagemap_kernel, dim3(Bq), dim3(kTopkThreads), smem, stream, a);
+  }
+  cudaError_t e = set_smem_once<topk_gather_kernel>(smem);
+  if (e == cudaSuccess) e = set_smem_once<topk_select_kernel>(smem);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(topk_gather_kernel, dim3(a.chunks, Bq), dim3(kTopkThreads), smem, stream, a);
+  ++*launches;
   if (e != cudaSuccess) return e;
   ++*launches;
-  return launch_pdl(topk_pagemap_kernel, dim3(Bq), dim3(kTopkThreads), smem, stream, a);
+  return launch_pdl(topk_select_kernel, dim3(Bq), dim3(kTopkThreads), smem, stream, a);
 }
 
 cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,

@@ -185,3 +185,19 @@ def test_topk_unaligned_rows():
     for i in range(3):
         check_topk_exact(lo[i], scores[i], vis[i], 512)
     assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
+
+
+def test_topk_long_rows_chunked_path():
+    """Rows of 200K keys take the chunked gather (one CTA per 16K keys, per-row candidates
+    in the workspace). The constant row overflows the candidate buffer and falls back to
+    the whole-row select; the random row is selected from its candidates."""
+    import deepseek_sparse_attention_head_b200 as dsa
+    rng = np.random.default_rng(6)
+    L = 200000
+    scores = np.stack([np.full(L, 0.75), rng.standard_normal(L)]).astype(np.float32)
+    vis = np.array([L, L - 1000])
+    case, lo, ph, err = _topk_on_scores(scores, vis, 2048)
+    assert err == 0
+    for i in range(2):
+        check_topk_exact(lo[i], scores[i], vis[i], 2048)
+    assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
