@@ -39,7 +39,9 @@ struct IdxCfg {
   static constexpr int kPagesPerTile = kTileTok / kPage;
   static constexpr int kBatch = 32 / kPagesPerTile;   // tiles whose block-table entries the producer fetches at once
   static constexpr int kHalves = kTileTok / 128;       // 128-token MMA halves (M = 128) per tile
-  static constexpr int kUnitHalves = QG == 1 ? 2 : 1;  // halves per accumulator unit (one commit, one wait)
+  // Decode: one accumulator unit per tile, signalled by the stage's own completion barrier
+  // (one wait and one commit per tile for the issuer). Prefill: one unit per half and query group.
+  static constexpr int kUnitHalves = QG == 1 ? kHalves : 1;
   static constexpr int kChunk = kTileTok * 128;        // one 128-byte K-chunk of a tile
   static constexpr int kStages = KC == 1 ? (QG == 1 ? 3 : 4) : 2;
   static constexpr int kBSlots = (KC == 2 && QG == 4) ? 1 : 2;
@@ -57,7 +59,7 @@ struct IdxCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
 };
-static_assert(IdxCfg<1, 1>::kHalves / IdxCfg<1, 1>::kUnitHalves == 2 &&
+static_assert(IdxCfg<1, 1>::kHalves / IdxCfg<1, 1>::kUnitHalves == 1 &&
                   IdxCfg<1, 4>::kHalves / IdxCfg<1, 4>::kUnitHalves == 2 &&
                   IdxCfg<2, 1>::kHalves / IdxCfg<2, 1>::kUnitHalves == 1,
               "units per tile");
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                     else mma_f16(d, ao, bo, idesc, (kc | ks) != 0);
                   }
               }
-              tc_commit(&acc_full[ab]);
+              if (QG != 1) tc_commit(&acc_full[ab]);   // decode: the stage commit below signals it
             }
             __syncwarp();
           }
@@ -420,7 +422,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               cur_q0 = q0;
             }
             const int ab = unit % n_acc;
-            if (!wait_warp(&acc_full[ab], (unit / n_acc) & 1, abort_flag)) { ok = false; break; }
+            // decode: unit == tile index, and the tile's stage barrier completes with its MMAs
+            const bool got = QG == 1 ? wait_warp(&a_empty[unit % C::kStages], (unit / C::kStages) & 1, abort_flag)
+                                     : wait_warp(&acc_full[ab], (unit / n_acc) & 1, abort_flag);
+            if (!got) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int hh = 0; hh < UH; ++hh) {
