@@ -151,8 +151,12 @@ def file_hash(paths):
     return h.hexdigest()[:16]
 
 
-INDEXER_SOURCES = ["deepseek_sparse_attention_head_b200/csrc/indexer.cu",
-                   "deepseek_sparse_attention_head_b200/csrc/common.cuh"]
+KERNEL_SOURCES = {
+    "indexer": ["deepseek_sparse_attention_head_b200/csrc/indexer.cu",
+                "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
+    "mla": ["deepseek_sparse_attention_head_b200/csrc/mla.cu",
+            "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
+}
 
 
 def measured_peaks():
@@ -168,13 +172,15 @@ def measured_peaks():
 FP8_OVER_BF16 = 2.0     # nominal dense tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
 
 
-def committed_traffic():
-    """Per-launch DRAM bytes of the indexer kernel from the committed ncu summary, or None
-    when the summary is absent or was taken on different kernel sources."""
+def committed_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from its committed ncu summary, or None when the
+    summary is absent, was taken on different kernel sources, or on another workload."""
     try:
-        with open(os.path.join(ROOT, "profiles", "indexer_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")) as f:
             d = json.load(f)
-        if d.get("sources_sha") != file_hash(INDEXER_SOURCES):
+        if d.get("sources_sha") != file_hash(KERNEL_SOURCES[kernel]):
+            return None
+        if not d.get("workload", "").startswith(workload + ":"):
             return None
         return d
     except (OSError, ValueError):
@@ -266,6 +272,31 @@ def run_ours(args, world, rank, local):
     e1.synchronize()
     idx_ms = e0.elapsed_time(e1) / reps
 
+    # ---- MLA stage timed alone on the selection a layer call made (decode + combine kernels)
+    phys = torch.empty(Bq, K, dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(stream):
+        dsa.dsa_decode_layer(paging, t["q_idx"], t["q_idx_scale"], t["head_w"], t["k_cache"], t["k_scale"],
+                             t["q_mla"], t["kv_cache"], t["kv_scale"], K, case["softmax_scale"], out, ws, lse=lse,
+                             physical_out=phys, stream=stream)
+    ws_m = dsa.alloc_workspace(dsa.mla_workspace_size(Bq, K))
+
+    def mla_call():
+        dsa.mla_sparse_decode(t["q_mla"], t["kv_cache"], t["kv_scale"], phys, case["softmax_scale"], out, lse, ws_m,
+                              stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            mla_call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            mla_call()
+        e1.record(stream)
+    e1.synchronize()
+    mla_ms = e0.elapsed_time(e1) / reps
+    if dsa.dsa_get_error(ws_m, stream) != 0:
+        raise RuntimeError("device error in the MLA timing calls")
+
     # ---- end to end through the public API with host buffers
     pin = {k: t[k].cpu().pin_memory() for k in ("q_idx", "q_idx_scale", "head_w", "q_mla", "seq_lens",
                                                    "block_table") if t[k] is not None}
@@ -291,24 +322,42 @@ def run_ours(args, world, rank, local):
 
     hbm_peak, bf16_peak, peak_kind = measured_peaks()
     calls_per_s = whole_job_rate(world, args.steps, ms_max)
-    tr = committed_traffic()
-    if tr is not None and not tr.get("workload", "").startswith(args.workload + ":"):
-        tr = None                      # the committed capture is of another workload
-    if case["n_q"] > 1:
-        # chunked prefill: the indexer contraction is tensor-bound (fp8 x fp8)
-        flops = dsa_inputs.indexer_flops(case)
-        achieved = flops / (idx_ms / 1e3) / 1e12
-        peak = bf16_peak * FP8_OVER_BF16
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak,
-                    "peak_kind": f"{peak_kind} bf16_tflops (burst) x {FP8_OVER_BF16:g} nominal fp8/bf16 ratio",
-                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None, "algorithmic_flops": flops}
-    else:
-        achieved = nbytes["indexer"] / (idx_ms / 1e3) / 1e9
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-                    "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "unit": "GB/s", "frac": achieved / hbm_peak,
-                    "traffic": None if tr is None else tr["bytes_per_launch"], "algorithmic_bytes": nbytes["indexer"]}
-    roofline["kernel"] = "indexer (dsa_indexer_scores call: plan + tcgen05 indexer)"
-    roofline["duration_us"] = idx_ms * 1e3
+
+    def roofline_of(name, call, ms, nb, flops, flop_peak, flop_kind):
+        """Bound = whichever of HBM bytes and tensor FLOPs gives the longer ideal time."""
+        t_hbm = nb / (hbm_peak * 1e9)
+        t_tc = flops / (flop_peak * 1e12)
+        if t_tc > t_hbm:
+            ach = flops / (ms / 1e3) / 1e12
+            r = {"bound": "tensor", "achieved": ach, "peak": flop_peak, "peak_kind": flop_kind, "unit": "TFLOP/s",
+                 "frac": ach / flop_peak, "traffic": None, "algorithmic_flops": flops}
+        else:
+            ach = nb / (ms / 1e3) / 1e9
+            tr = committed_traffic(name, args.workload)
+            r = {"bound": "hbm", "achieved": ach, "peak": hbm_peak,
+                 "peak_kind": f"{peak_kind} hbm_gbs (burst copy)", "unit": "GB/s", "frac": ach / hbm_peak,
+                 "traffic": None if tr is None else tr["bytes_per_launch"], "algorithmic_bytes": nb}
+        r["kernel"] = call
+        r["duration_us"] = ms * 1e3
+        return r
+
+    # indexer: keys (+ scales, block table) and queries; fp8 x fp8 contraction
+    idx_flops = dsa_inputs.indexer_flops(case)
+    fp8 = case["idx_dtype"] != "bf16"
+    idx_peak = bf16_peak * (FP8_OVER_BF16 if fp8 else 1.0)
+    idx_kind = (f"{peak_kind} bf16_tflops (burst) x {FP8_OVER_BF16:g} nominal fp8/bf16 ratio" if fp8
+                else f"{peak_kind} bf16_tflops (burst)")
+    rf_idx = roofline_of("indexer", "indexer (dsa_indexer_scores call: plan + tcgen05 indexer)", idx_ms,
+                         nbytes["indexer"], idx_flops, idx_peak, idx_kind)
+    # MLA: selected latent rows, bf16 queries and the output; QK (576) + PV (512) per selected row
+    sel = int(np.minimum(dsa_inputs.vis_lengths(case), K).sum())
+    out_b = 4 if case["out_dtype"] == "fp32" else 2
+    mla_bytes = nbytes["mla"] + Bq * (2 * 64 * 576 + out_b * 64 * 512)
+    mla_flops = 2 * sel * 64 * (576 + 512)
+    rf_mla = roofline_of("mla", "mla (mla_sparse_decode call: tcgen05 MLA decode + split combine)", mla_ms,
+                         mla_bytes, mla_flops, bf16_peak, f"{peak_kind} bf16_tflops (burst)")
+    # the dominant kernel is the one that takes longer
+    roofline, other = (rf_mla, rf_idx) if mla_ms > idx_ms else (rf_idx, rf_mla)
     result = {
         "metric": METRIC,
         "value": calls_per_s,
@@ -332,6 +381,7 @@ def run_ours(args, world, rank, local):
         },
         "achieved_hbm_tbs": nbytes["total"] / (ms_max / args.steps / 1e3) / 1e12,
         "roofline": roofline,
+        "roofline_other_kernel": other,
         "e2e": {"value": world * n_e2e / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": n_e2e},
         "gpu_launches": launches_per_step * args.steps,
