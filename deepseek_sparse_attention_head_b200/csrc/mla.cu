@@ -123,6 +123,20 @@ __device__ __forceinline__ float ex2_ftz(float x) {  // hardware 2^x; tiny resul
   return y;
 }
 
+// Read-only global loads that write their destination only when `pred` holds (it keeps
+// the value it had otherwise), so that nothing after the load has to wait for it to
+// choose between the loaded value and a default.
+__device__ __forceinline__ void ldg_pred(uint4& v, const void* p, bool pred) {
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}\n"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
+      : "l"(p), "r"(static_cast<uint32_t>(pred)));
+}
+__device__ __forceinline__ void ldg_pred(float& v, const float* p, bool pred) {
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q ld.global.nc.f32 %0, [%1];\n\t}\n"
+      : "+f"(v)
+      : "l"(p), "r"(static_cast<uint32_t>(pred)));
+}
+
 // Four E4M3 codes -> four fp16 (exact) times the fp16 multiplier pair m2.
 __device__ __forceinline__ void dequant4_f16(uint32_t w, __half2 m2, uint32_t& o0, uint32_t& o1) {
   const __half2_raw r01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
@@ -542,26 +556,28 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       for (int i = 0; i < kBatchPieces; ++i) {
         const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
         const int c16 = p % kRowPieces;
-        raw[i] = sl[i] >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.kv + static_cast<int64_t>(sl[i]) * kRowBytes) + c16)
-                            : make_uint4(0u, 0u, 0u, 0u);
+        raw[i] = make_uint4(0u, 0u, 0u, 0u);
+        ldg_pred(raw[i], a.kv + static_cast<int64_t>(max(sl[i], 0)) * kRowBytes + c16 * 16, sl[i] >= 0);
       }
     };
     auto fetch_meta = [&](float (&sc)[kKvGroups], int& my_slot, int T) {
       if (lt < kMlaTile) {
         my_slot = slot_at(T, lt);
 #pragma unroll
-        for (int k = 0; k < kKvGroups; ++k)
-          sc[k] = (FP8 && my_slot >= 0) ? __ldg(a.kv_scale + static_cast<int64_t>(my_slot) * kKvGroups + k) : 0.0f;
+        for (int k = 0; k < kKvGroups; ++k) {
+          sc[k] = 0.0f;
+          if (FP8) ldg_pred(sc[k], a.kv_scale + static_cast<int64_t>(max(my_slot, 0)) * kKvGroups + k, my_slot >= 0);
+        }
       }
     };
     auto store = [&](const uint4 (&raw)[kBatchPieces], int batch, uint8_t* kv, const uint32_t* mult) {
+      if (FP8) {
 #pragma unroll
-      for (int i = 0; i < kBatchPieces; ++i) {
-        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
-        const int row = p / kRowPieces, c16 = p - row * kRowPieces;
-        if (FP8) {
-          const uint32_t mw = mult[row * kKvGroups + (c16 >> 3)];
-          const __half2 m2 = *reinterpret_cast<const __half2*>(&mw);
+        for (int i = 0; i < kBatchPieces; ++i) {
+          const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+          const int row = p / kRowPieces, c16 = p - row * kRowPieces;
+          const uint32_t mwi = mult[row * kKvGroups + (c16 >> 3)];
+          const __half2 m2 = *reinterpret_cast<const __half2*>(&mwi);
           uint4 o0, o1;
           dequant4_f16(raw[i].x, m2, o0.x, o0.y);
           dequant4_f16(raw[i].y, m2, o0.z, o0.w);
@@ -569,15 +585,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           dequant4_f16(raw[i].w, m2, o1.z, o1.w);
           uint8_t* blk = kv + (c16 >> 2) * kKVChunk;
           const int u = (c16 & 3) * 2;
-          // alternate which half goes first by chunk parity: spreads a warp's stores over banks
-          if ((c16 >> 2) & 1) {
-            *reinterpret_cast<uint4*>(blk + swz(row, u + 1)) = o1;
-            *reinterpret_cast<uint4*>(blk + swz(row, u)) = o0;
-          } else {
-            *reinterpret_cast<uint4*>(blk + swz(row, u)) = o0;
-            *reinterpret_cast<uint4*>(blk + swz(row, u + 1)) = o1;
-          }
-        } else {
+          // odd chunks store their upper half first, which spreads each store instruction
+          // of a warp over all eight 16-byte bank groups; chosen by selects, not a branch
+          const int odd = (c16 >> 2) & 1;
+          const uint4 first = odd ? o1 : o0;
+          const uint4 second = odd ? o0 : o1;
+          *reinterpret_cast<uint4*>(blk + swz(row, u + odd)) = first;
+          *reinterpret_cast<uint4*>(blk + swz(row, u + 1 - odd)) = second;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kBatchPieces; ++i) {
+          const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+          const int row = p / kRowPieces, c16 = p - row * kRowPieces;
           *reinterpret_cast<uint4*>(kv + (c16 >> 3) * kKVChunk + swz(row, c16 & 7)) = raw[i];
         }
       }
