@@ -8,7 +8,7 @@
 //     a margin) lie above it.
 //  2. One pass over the row gathers every key at or above the threshold into shared
 //     memory (per-thread counts, a warp prefix sum and one shared atomic per warp for
-//     every 16K keys).
+//     every 16K keys). Its first batch is loaded before step 1 starts.
 //  3. The k-th largest candidate is found exactly by a radix select over the
 //     candidates' offsets from the threshold (12-bit digits, shared-memory
 //     histograms), and the winners are emitted with their physical slots.
@@ -237,42 +237,65 @@ __device__ uint32_t row_threshold_small(TopkSmem& sm, const float* row, int vis,
   return thr;
 }
 
+constexpr int kGatherU = 16;                               // keys per thread and batch
+constexpr int kGatherBatch = kGatherU * kTopkThreads;
+
+// Loads the gather batch of row[base, hi_s) that starts at `base` (a multiple of 4, the
+// row 16-byte aligned): thread t gets keys base + 4 (j * 1024 + t) + [0, 4), j < 4, zeros
+// past hi_s. A whole batch in range takes plain 16-byte loads (CTA-uniform test).
+__device__ __forceinline__ void gather_load(const float* row, int base, int hi_s, float4 (&v)[kGatherU / 4]) {
+  const int tid = threadIdx.x;
+  const float4* r4 = reinterpret_cast<const float4*>(row);
+  if (base + kGatherBatch <= hi_s) {
+#pragma unroll
+    for (int j = 0; j < kGatherU / 4; ++j) v[j] = __ldg(r4 + (base >> 2) + j * kTopkThreads + tid);
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < kGatherU / 4; ++j) {
+    const int s_ = base + 4 * (j * kTopkThreads + tid);
+    v[j] = s_ + 3 < hi_s ? __ldg(r4 + (s_ >> 2))
+                         : make_float4(s_ < hi_s ? row[s_] : 0.0f, s_ + 1 < hi_s ? row[s_ + 1] : 0.0f,
+                                       s_ + 2 < hi_s ? row[s_ + 2] : 0.0f, 0.0f);
+  }
+}
+
+// Bit 4 j + t set when key t of cur[j] (index base + 4 (j * 1024 + tid) + t) is below
+// hi_s (checked unless kWhole) and at least thr.
+template <bool kWhole>
+__device__ __forceinline__ uint32_t gather_takes(const float4 (&cur)[kGatherU / 4], int base, int hi_s,
+                                                 uint32_t thr) {
+  uint32_t takes = 0;
+#pragma unroll
+  for (int j = 0; j < kGatherU / 4; ++j) {
+    const int s_ = base + 4 * (j * kTopkThreads + static_cast<int>(threadIdx.x));
+    const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if ((kWhole || s_ + t < hi_s) && order_key(e[t]) >= thr) takes |= 1u << (4 * j + t);
+  }
+  return takes;
+}
+
 // Gathers every key >= thr of row[lo_s, hi_s) (lo_s a multiple of 4, the row 16-byte
 // aligned) into out_key / out_idx at slots reserved from *counter (shared or global; one
 // atomic per warp per 16K keys; slots >= cap are counted but not stored), and raises
-// *rmax_addr to the largest key - thr. Whole CTA; the trip count is CTA-uniform.
+// *rmax_addr to the largest key - thr. `cur` holds the first batch, loaded by
+// gather_load(row, lo_s, hi_s, cur) (so that its loads can be in flight while the caller
+// derives thr). Whole CTA; the trip count is CTA-uniform.
 __device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr, uint32_t* counter,
-                             uint32_t* out_key, int32_t* out_idx, uint32_t cap, uint32_t* rmax_addr) {
-  constexpr int kU = 16;
-  constexpr int kBatch = kU * kTopkThreads;
+                             uint32_t* out_key, int32_t* out_idx, uint32_t cap, uint32_t* rmax_addr,
+                             float4 (&cur)[kGatherU / 4]) {
   const int tid = threadIdx.x;
-  const float4* r4 = reinterpret_cast<const float4*>(row);
-  auto load_batch = [&](int base, float4 (&v)[kU / 4]) {
-#pragma unroll
-    for (int j = 0; j < kU / 4; ++j) {
-      const int s_ = base + 4 * (j * kTopkThreads + tid);
-      v[j] = s_ + 3 < hi_s ? __ldg(r4 + (s_ >> 2))
-                           : make_float4(s_ < hi_s ? row[s_] : 0.0f, s_ + 1 < hi_s ? row[s_ + 1] : 0.0f,
-                                         s_ + 2 < hi_s ? row[s_ + 2] : 0.0f, 0.0f);
-    }
-  };
   uint32_t lmax = 0;
-  float4 cur[kU / 4], nxt[kU / 4];
-  load_batch(lo_s, cur);
-  for (int base = lo_s; base < hi_s; base += kBatch) {
-    if (base + kBatch < hi_s) load_batch(base + kBatch, nxt);
-    uint32_t takes = 0;
-#pragma unroll
-    for (int j = 0; j < kU / 4; ++j) {
-      const int s_ = base + 4 * (j * kTopkThreads + tid);
-      const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        if (s_ + t < hi_s && order_key(e[t]) >= thr) takes |= 1u << (4 * j + t);
-    }
+  float4 nxt[kGatherU / 4];
+  for (int base = lo_s; base < hi_s; base += kGatherBatch) {
+    if (base + kGatherBatch < hi_s) gather_load(row, base + kGatherBatch, hi_s, nxt);
+    const uint32_t takes = base + kGatherBatch <= hi_s ? gather_takes<true>(cur, base, hi_s, thr)
+                                                        : gather_takes<false>(cur, base, hi_s, thr);
     uint32_t c = warp_reserve(counter, static_cast<uint32_t>(__popc(takes)));
 #pragma unroll
-    for (int j = 0; j < kU / 4; ++j) {
+    for (int j = 0; j < kGatherU / 4; ++j) {
       const int s_ = base + 4 * (j * kTopkThreads + tid);
       const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
 #pragma unroll
@@ -289,7 +312,7 @@ __device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr,
       }
     }
 #pragma unroll
-    for (int j = 0; j < kU / 4; ++j) cur[j] = nxt[j];
+    for (int j = 0; j < kGatherU / 4; ++j) cur[j] = nxt[j];
   }
   const uint32_t wmax = __reduce_max_sync(0xffffffffu, lmax);
   if ((tid & 31) == 0 && wmax != 0u) atomicMax(rmax_addr, wmax);
@@ -478,13 +501,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
   // The sampled path needs 16-byte aligned rows (always true for the fused layer, whose
   // row stride is a multiple of 64); other rows take the whole-row radix select.
   if ((reinterpret_cast<uintptr_t>(rw.row) & 15) == 0) {
+    float4 first[kGatherU / 4];
+    gather_load(rw.row, 0, rw.vis, first);   // in flight while the threshold is derived
     const uint32_t thr = row_threshold_small(sm, rw.row, rw.vis, rw.K);
     if (threadIdx.x == 0) {
       sm.n_cand = 0;
       sm.rmax = 0;
     }
     __syncthreads();
-    gather_range(rw.row, 0, rw.vis, thr, &sm.n_cand, sm.cand_key, sm.cand_idx, kCand, &sm.rmax);
+    gather_range(rw.row, 0, rw.vis, thr, &sm.n_cand, sm.cand_key, sm.cand_idx, kCand, &sm.rmax, first);
     __syncthreads();
     const uint32_t n_c = sm.n_cand;
     if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand)) {
@@ -508,11 +533,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_gather_kernel(const TopkArg
   const int lo_s = static_cast<int>(blockIdx.x) * kTopkChunk;
   if (lo_s >= rw.vis) return;
   const int hi_s = min(rw.vis, lo_s + kTopkChunk);
+  float4 first[kGatherU / 4];
+  gather_load(rw.row, lo_s, hi_s, first);   // in flight while the threshold is derived
   const uint32_t thr = row_threshold(sm, rw.row, rw.vis, rw.K);
   const int64_t q = rw.q;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.g_thr[q] = thr;
   gather_range(rw.row, lo_s, hi_s, thr, a.g_cnt + q, a.g_key + q * a.cand_cap, a.g_idx + q * a.cand_cap,
-               static_cast<uint32_t>(a.cand_cap), a.g_rmax + q);
+               static_cast<uint32_t>(a.cand_cap), a.g_rmax + q, first);
 }
 
 // Long rows, part 2: one CTA per query selects exactly among the gathered candidates
