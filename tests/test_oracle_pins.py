@@ -48,6 +48,38 @@ def test_bf16_decode_vs_torch():
     assert np.array_equal(oracle.decode_bf16(bits), ref)
 
 
+def test_scales_apply_to_their_columns():
+    """The storage reading for fp8 tensors. Latent rows carry five scales: columns
+    [0,128), [128,256), [256,384), [384,512) and the 64 rope columns [512,576). Indexer
+    keys carry one scale per token, indexer queries one per (query, head). Codes are
+    decoded by PyTorch; the column ranges are written out by hand."""
+    rng = np.random.default_rng(3)
+    case = blank_case((64,), idx_dtype="fp8", kv_dtype="fp8")
+    codes = rng.integers(0, 256, size=(64, DK)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C                       # no NaN codes
+    case["kv_cache"][:64] = codes
+    scales = np.array([0.5, 2.0, 4.0, 8.0, 16.0], dtype=np.float32)
+    case["kv_scale"][:64] = scales
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.dequant_latent_rows(case, np.arange(64))
+    for g, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 384), (384, 512), (512, 576)]):
+        assert np.array_equal(got[:, lo:hi], vals[:, lo:hi] * float(scales[g])), g
+
+    kc = rng.integers(0, 0x7F, size=(64, DI)).astype(np.uint8)
+    case["k_cache"][0] = kc
+    case["k_scale"][0] = np.arange(1, 65, dtype=np.float32)
+    kv = torch.from_numpy(kc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got_k = oracle.dequant_index_keys(case, np.arange(64))
+    assert np.array_equal(got_k, kv * np.arange(1, 65, dtype=np.float64)[:, None])
+
+    qc = rng.integers(0, 0x7F, size=(H, DI)).astype(np.uint8)
+    case["q_idx"][0] = qc
+    case["q_idx_scale"][0] = np.linspace(0.25, 4.0, H).astype(np.float32)
+    qv = torch.from_numpy(qc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got_q = oracle.dequant_index_queries(case)[0]
+    assert np.array_equal(got_q, qv * case["q_idx_scale"][0].astype(np.float64)[:, None])
+
+
 # ---------------------------------------------------------------- indexer
 
 def _worked_indexer_case(golden):
