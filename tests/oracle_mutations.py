@@ -122,6 +122,54 @@ def _combine_wrong_sign(ms, ls, os_):
     return out, lse
 
 
+def _visible_lengths_causal_off_by_one(case):
+    if case.get("q_pos") is not None:
+        return case["q_pos"].astype(np.int64)
+    return np.repeat(case["seq_lens"].astype(np.int64), case["n_q"])
+
+
+def _physical_slots_without_page_size(block_table_row, logical):
+    logical = np.asarray(logical, dtype=np.int64)
+    out = np.full(logical.shape, -1, dtype=np.int64)
+    ok = logical >= 0
+    li = logical[ok]
+    out[ok] = block_table_row[li // PAGE].astype(np.int64) + li % PAGE
+    return out
+
+
+def _mla_softmax_over_heads(case, physical, queries=None):
+    queries = np.arange(physical.shape[0]) if queries is None else np.asarray(queries)
+    scale = float(case["softmax_scale"])
+    out = np.zeros((len(queries), H, DV))
+    lse = np.full((len(queries), H), -np.inf)
+    for i, q in enumerate(queries):
+        sel = physical[i][physical[i] >= 0]
+        if sel.size == 0:
+            continue
+        qm = od.decode_bf16(case["q_mla"][q])
+        KV = od.dequant_latent_rows(case, sel)
+        z = scale * (qm @ KV.T)                                  # [64 heads, n keys]
+        m = z.max(axis=0, keepdims=True)                         # normalised over heads
+        e = np.exp(z - m)
+        l = e.sum(axis=0, keepdims=True)
+        out[i] = (e / l) @ KV[:, :DV]
+        lse[i] = np.log(np.exp(z).sum(axis=1))
+    return out, lse
+
+
+def _combine_without_l(ms, ls, os_):
+    ms, ls, os_ = np.stack(ms), np.stack(ls), np.stack(os_)
+    M = ms.max(axis=0)
+    Msafe = np.where(np.isfinite(M), M, 0.0)
+    a = np.where(np.isfinite(ms), np.exp(ms - Msafe[None, :]), 0.0)
+    L = a.sum(axis=0)                                            # the l_s weights are missing
+    O = (a[:, :, None] * os_).sum(axis=0)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where(L[:, None] > 0, O / np.where(L > 0, L, 1.0)[:, None], 0.0)
+        lse = np.where(L > 0, Msafe + np.log(np.where(L > 0, L, 1.0)), -np.inf)
+    return out, lse
+
+
 def _bf16_shift15(bits):
     b = np.asarray(bits).astype(np.uint32) << np.uint32(15)
     return b.view(np.float32).astype(np.float64)
@@ -153,6 +201,10 @@ MUTATIONS = {
     "mla_keys_without_rope_columns": lambda: _set("mla_sparse_attention", _mla(key_cols=slice(0, DV))),
     "mla_lse_without_the_max": lambda: _set("mla_sparse_attention", _mla(lse_with_max=False)),
     "combine_weights_with_wrong_sign": lambda: _set("combine_partials", _combine_wrong_sign),
+    "combine_without_the_normalisers": lambda: _set("combine_partials", _combine_without_l),
+    "causal_visibility_off_by_one": lambda: _set("visible_lengths", _visible_lengths_causal_off_by_one),
+    "pagemap_without_the_page_size": lambda: _set("physical_slots", _physical_slots_without_page_size),
+    "mla_softmax_over_heads": lambda: _set("mla_sparse_attention", _mla_softmax_over_heads),
 }
 
 
