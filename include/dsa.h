@@ -25,8 +25,8 @@
  *    a sequence longer than its block-table row, a slot index outside the cache)
  *    are clamped so no access leaves its buffer, and are recorded in a sticky error
  *    word inside the workspace; read it with dsa_get_error(). Kernels never trap.
- *    Every wait inside a kernel is bounded (about one second); a wait that runs out
- *    records DSA_ERR_TIMEOUT and the kernel returns.
+ *    Every wait inside a kernel is bounded (4e9 SM clock cycles, about two seconds); a
+ *    wait that runs out records DSA_ERR_TIMEOUT and the kernel returns.
  *  - The workspace must be zero-filled once before its first use (cudaMemset); the
  *    library leaves it reusable. Calls sharing one workspace must be stream-ordered.
  *  - Layouts are row-major and contiguous as annotated. "fp8" is OCP FP8 E4M3, the
@@ -156,8 +156,8 @@ dsa_status mla_sparse_decode(int32_t Bq, const void* q, const void* kv_cache, ds
  * mla_sparse_decode without a workspace argument, for callers that cannot allocate
  * device memory themselves: a plugin running inside an engine that reserves and owns all
  * of the GPU's memory and hands out none of it, or a decode loop that must not call
- * cudaMalloc and cudaFree, which can synchronise the whole device. The paper has no counterpart to this entry point; it is a packaging of
- * stage 3 only. Arguments and results are those of mla_sparse_decode, except:
+ * cudaMalloc and cudaFree, which can synchronise the whole device. The source pages
+ * have no counterpart to this entry point; it is a packaging of stage 3 only. Arguments and results are those of mla_sparse_decode, except:
  *  status  optional device [2] uint32 (8-byte aligned), or NULL: receives this call's
  *          device-side error words; read and clear it with dsa_get_error(status, stream).
  *          With NULL, device-side range and timeout errors are not reported.
