@@ -117,7 +117,8 @@ dsa_status dsa_indexer_scores(const dsa_paging* paging,
  *  physical_out device [B*n_q, top_k] int32 physical slots block_table[b,s/64]*64+s%64
  * Entries k..top_k-1 are -1. Equal scores at the boundary are broken arbitrarily.
  * Scores are ranked by the IEEE-754 total order of their bit patterns
- * (-NaN < -inf < ... < -0 < +0 < ... < +inf < +NaN); dsa_indexer_scores writes no NaN.
+ * (-NaN < -inf < ... < -0 < +0 < ... < +inf < +NaN); dsa_indexer_scores writes no NaN
+ * when its inputs are finite.
  *  scores  device [B*n_q, L_max] fp32 (as written by dsa_indexer_scores)
  *  1 <= top_k <= 16384.
  */
