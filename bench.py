@@ -157,6 +157,7 @@ KERNEL_SOURCES = {
     "indexer": ["deepseek_sparse_attention_head_b200/csrc/indexer.cu",
                 "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
     "mla": ["deepseek_sparse_attention_head_b200/csrc/mla.cu",
+            "deepseek_sparse_attention_head_b200/csrc/mla_fp8.cu",
             "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
 }
 
@@ -172,6 +173,31 @@ def measured_peaks():
 
 
 FP8_OVER_BF16 = 2.0     # nominal dense tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
+
+
+def measure_fp8_peak(stream, n=8192, reps=30):
+    """Dense e4m3 tensor-core throughput of this GPU, measured like the bf16 entry of
+    MEASURED_PEAKS.json: a large library GEMM (torch._scaled_mm, e4m3 x e4m3 -> bf16,
+    n x n x n, per-tensor scales) timed as a burst of back-to-back calls with CUDA events.
+    Returns (TFLOP/s, description) or (None, reason)."""
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        del a, b
+        return 2.0 * n ** 3 / (ms / 1e3) / 1e12, f"torch._scaled_mm e4m3 {n}^3 -> bf16, burst of {reps}, CUDA events"
+    except Exception as exc:  # noqa: BLE001 - reported in the JSON line, not fatal
+        return None, f"fp8 GEMM unavailable: {type(exc).__name__}"
 
 
 def committed_traffic(kernel: str, workload: str):
@@ -334,13 +360,34 @@ def run_ours(args, world, rank, local):
     d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
     n_e2e = max(10, args.e2e_steps)
 
-    def e2e_step():
+    def e2e_body():
         for k, v in pin.items():
             t[k].copy_(v, non_blocking=True)
         step()
         host_out.copy_(out, non_blocking=True)
         host_lse.copy_(lse, non_blocking=True)
 
+    # the whole step, host copies included, replayed from one CUDA graph (as a serving loop
+    # would run it); eager launches when graphs are off
+    e2e_graph = None
+    if graph is not None:
+        with torch.cuda.stream(stream):
+            e2e_body()
+        stream.synchronize()
+        e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e2e_graph, stream=stream):
+            e2e_body()
+        stream.synchronize()
+
+    def e2e_step():
+        if e2e_graph is not None:
+            e2e_graph.replay()
+        else:
+            e2e_body()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
     barrier(world)
     torch.cuda.synchronize()
     if inputs_exceed_l2:
@@ -374,9 +421,15 @@ def run_ours(args, world, rank, local):
     # indexer: keys (+ scales, block table) and queries; fp8 x fp8 contraction
     idx_flops = dsa_inputs.indexer_flops(case)
     fp8 = case["idx_dtype"] != "bf16"
-    idx_peak = bf16_peak * (FP8_OVER_BF16 if fp8 else 1.0)
-    idx_kind = (f"{peak_kind} bf16_tflops (burst) x {FP8_OVER_BF16:g} nominal fp8/bf16 ratio" if fp8
-                else f"{peak_kind} bf16_tflops (burst)")
+    fp8_peak, fp8_how = (None, "not measured (the indexer is HBM-bound here)")
+    if fp8 and idx_flops / (bf16_peak * FP8_OVER_BF16 * 1e12) > nbytes["indexer"] / (hbm_peak * 1e9):
+        fp8_peak, fp8_how = measure_fp8_peak(stream)    # tensor-bound (chunked prefill): measure it
+    if fp8 and fp8_peak is not None:
+        idx_peak, idx_kind = fp8_peak, f"measured fp8 peak ({fp8_how})"
+    else:
+        idx_peak = bf16_peak * (FP8_OVER_BF16 if fp8 else 1.0)
+        idx_kind = (f"{peak_kind} bf16_tflops (burst) x {FP8_OVER_BF16:g} nominal fp8/bf16 ratio" if fp8
+                    else f"{peak_kind} bf16_tflops (burst)")
     rf_idx = roofline_of("indexer", "indexer (dsa_indexer_scores call: plan + tcgen05 indexer)", idx_ms,
                          nbytes["indexer"], idx_flops, idx_peak, idx_kind, idx_how)
     # MLA: selected latent rows, bf16 queries and the output; QK (576) + PV (512) per selected row
@@ -398,7 +451,8 @@ def run_ours(args, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": (f"{'bf16' if case['idx_dtype'] == 'bf16' else 'e4m3'} indexer + "
-                  f"{'bf16' if case['kv_dtype'] == 'bf16' else 'f16'} MLA operands, fp32 accumulate"),
+                  f"{'bf16' if case['kv_dtype'] == 'bf16' else 'e4m3 (two-term queries and weights)'} MLA "
+                  f"operands, fp32 accumulate"),
         "data": "synthetic (seeded; dsa_inputs)",
         "config": {
             "workload": f"{args.workload}: {dsa_inputs.WORKLOAD_NAMES[args.workload]}",
@@ -415,12 +469,17 @@ def run_ours(args, world, rank, local):
         "roofline": roofline,
         "roofline_other_kernel": other,
         "e2e": {"value": world * n_e2e / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": n_e2e},
+                "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                "launch": "cuda_graph (copies included)" if e2e_graph is not None else "eager"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if fp8_peak is not None:
+        result["fp8_tensor_peak"] = {"tflops": fp8_peak, "how": fp8_how}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(case, budget_s=20.0)
+    if e2e_graph is not None:
+        del e2e_graph
     if graph is not None:
         del graph
     return result
@@ -451,12 +510,22 @@ def time_oracle_rows(case, rows, deadline=None):
 
 def cpu_baseline(case, budget_s=20.0):
     """The oracle as it stands on this host's cores, on whole query rows of the workload
-    until about budget_s of CPU work; scaled to layer-calls/s by the row count."""
+    until about budget_s of CPU work; scaled to layer-calls/s by the row count. A second,
+    shorter sample runs the same oracle on one core (BLAS limited to one thread)."""
     rows = list(range(case["Bq"]))
     dt, done = time_oracle_rows(case, rows, deadline=budget_s)
     per_row = dt / done
-    return {"value": 1.0 / (per_row * case["Bq"]), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{done} of {case['Bq']} query rows (full indexer+top-k+MLA per row), {dt:.1f} s"}
+    res = {"value": 1.0 / (per_row * case["Bq"]), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+           "sample": f"{done} of {case['Bq']} query rows (full indexer+top-k+MLA per row), {dt:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            dt1, done1 = time_oracle_rows(case, rows[:max(1, done // 4)], deadline=budget_s / 2)
+        res["single_core"] = {"value": 1.0 / (dt1 / done1 * case["Bq"]), "unit": UNIT, "cores": 1,
+                              "sample": f"{done1} query rows, {dt1:.1f} s"}
+    except ImportError:
+        pass
+    return res
 
 
 def run_reference(args, world, rank):

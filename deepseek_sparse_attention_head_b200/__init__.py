@@ -69,6 +69,7 @@ _SIGNATURES = {
     "dsa_get_error": (_i32, [_vp, _vp]),
     "dsa_status_string": (ctypes.c_char_p, [_i32]),
     "dsa_last_launch_count": (_i32, []),
+    "dsa_test_set_wait_hooks": (_i32, [_i64, _i32]),
 }
 
 
@@ -131,6 +132,12 @@ def dsa_status_string(status: int) -> str:
 
 def dsa_last_launch_count() -> int:
     return int(_lib.dsa_last_launch_count())
+
+
+def dsa_test_set_wait_hooks(wait_limit_cycles: int = 0, stall: bool = False):
+    """Test hook of the fp8-cache MLA kernel's bounded waits (this host thread's later
+    calls): a shorter wait bound, and optionally a wait that nothing satisfies."""
+    _check(_lib.dsa_test_set_wait_hooks(int(wait_limit_cycles), 1 if stall else 0), "dsa_test_set_wait_hooks")
 
 
 class Paging:

@@ -14,6 +14,9 @@ using namespace dsa;
 namespace {
 
 thread_local int g_launches = 0;
+// test hooks of dsa_test_set_wait_hooks (this host thread's later MLA launches)
+thread_local long long g_test_wait_limit = 0;
+thread_local int g_test_stall = 0;
 
 // ------------------------------------------------------------------ device facts
 
@@ -126,7 +129,7 @@ Layout layout_for(int B, int64_t Bq, int64_t L_max, int top_k, int op, int nspli
   }
   if ((op == DSA_OP_LAYER || op == -1) && nsplit > 1) {
     l.part_ml = off;
-    off += up256(static_cast<size_t>(Bq) * nsplit * kHeads * 2 * 4);
+    off += up256(static_cast<size_t>(Bq) * nsplit * kHeads * kPartStats * 4);
     l.part_o = off;
     off += up256(static_cast<size_t>(Bq) * nsplit * kHeads * kDimV * 4);
   }
@@ -227,6 +230,7 @@ dsa_status run_mla(int Bq, const void* q, const void* kv, dsa_dtype kv_dtype, co
   if (!make_map(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDimK, static_cast<uint64_t>(Bq) * kHeads, 64, 64))
     return DSA_ERR_CUDA;
   MlaArgs a;
+  a.q = q;
   a.Bq = Bq;
   a.top_k = top_k;
   a.nsplit = nsplit;
@@ -242,6 +246,8 @@ dsa_status run_mla(int Bq, const void* q, const void* kv, dsa_dtype kv_dtype, co
   a.part_ml = nsplit > 1 ? reinterpret_cast<float*>(ws + lay.part_ml) : nullptr;
   a.part_o = nsplit > 1 ? reinterpret_cast<float*>(ws + lay.part_o) : nullptr;
   a.err = err_word(ws);
+  a.wait_limit = g_test_wait_limit > 0 ? g_test_wait_limit : kWaitLimitCycles;
+  a.stall = g_test_stall;
   return cuda_status(launch_mla(kv_dtype == DSA_FP8_E4M3, tq, a, st, &g_launches));
 }
 
@@ -442,6 +448,13 @@ const char* dsa_status_string(dsa_status status) {
 }
 
 int32_t dsa_last_launch_count(void) { return g_launches; }
+
+dsa_status dsa_test_set_wait_hooks(int64_t wait_limit_cycles, int32_t stall) {
+  if (wait_limit_cycles < 0 || (stall != 0 && stall != 1)) return DSA_ERR_INVALID_ARG;
+  g_test_wait_limit = wait_limit_cycles;
+  g_test_stall = stall;
+  return DSA_OK;
+}
 
 }  // extern "C"
 

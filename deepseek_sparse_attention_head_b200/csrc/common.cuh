@@ -76,16 +76,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Single-thread bounded wait. Returns false when the bound ran out or another role
-// raised `abort_flag`; the caller then records DSA_ERR_TIMEOUT and unwinds.
-__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Single-thread bounded wait. Returns false when `limit` SM cycles ran out or another
+// role raised `abort_flag`; the caller then records DSA_ERR_TIMEOUT and unwinds.
+__device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) return false;
+      if (clock64() - t0 > limit) return false;
     }
   }
 }
@@ -93,12 +94,13 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatil
 // Warp-uniform bounded wait. Every lane tests the phase once (one round trip when it has
 // already completed, the common case); otherwise lane 0 polls alone and the other lanes
 // confirm afterwards, so a waiting warp issues few barrier operations.
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit = kWaitLimitCycles) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, abort_flag);
+  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, abort_flag, limit);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-  if (ok) ok = wait_one(bar, parity, abort_flag);
+  if (ok) ok = wait_one(bar, parity, abort_flag, limit);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -151,6 +153,60 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 16-byte global -> shared copy through L2 (cp.async, no register staging). With
+// src_bytes = 0 nothing is read and the 16 bytes are zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// 4-byte variant (cached at L1 and L2); src_bytes = 0 zero-fills.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrives once on `bar` when every cp.async this thread issued before has completed; the
+// arrival counts against the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// bar.red over named barrier `id` of `count` threads: OR / AND of a predicate. Also a
+// barrier: shared-memory writes before it are visible to the participants after it.
+__device__ __forceinline__ int bar_or(int id, int count, int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.or.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return static_cast<int>(r);
+}
+__device__ __forceinline__ int bar_and(int id, int count, int v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.and.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return static_cast<int>(r);
+}
+
+__device__ __forceinline__ int float_exponent(float s) {  // floor(log2 s) for positive normal s
+  return static_cast<int>((__float_as_uint(s) >> 23) & 0xFF) - 127;
+}
+
+__device__ __forceinline__ float exp2i(int e) {  // exact 2^e, clamped to the normal fp32 range
+  e = e < -126 ? -126 : (e > 127 ? 127 : e);
+  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
+}
+
+__device__ __forceinline__ float ex2_ftz(float x) {  // hardware 2^x; tiny results flush to zero
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -217,6 +273,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;   // descriptor version for tcgen05
   d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Same with 64-byte swizzle: 8-row atoms of 64-byte rows (16-byte chunk c of row r sits at
+// chunk c ^ ((r / 2) % 4)); K-major, sbo = 512 between 8-row groups.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;   // SWIZZLE_64B
   return d;
 }
 

@@ -47,7 +47,11 @@ struct TopkArgs {
   int32_t* g_idx;
 };
 
+// Per-(query, split, head) partial statistics: m, l, then one normaliser per value group.
+constexpr int kPartStats = 6;
+
 struct MlaArgs {
+  const void* q;        // [Bq, 64, 576] bf16 queries
   int Bq;
   int top_k;
   int nsplit;
@@ -60,9 +64,12 @@ struct MlaArgs {
   void* out;
   int out_fp32;
   float* lse;
-  float* part_ml;       // [Bq, nsplit, 64, 2]
+  float* part_ml;       // [Bq, nsplit, 64, kPartStats]: running max (log2 units), sum of p, and
+                        // the normaliser of each 128-column value group (see mla_combine_kernel)
   float* part_o;        // [Bq, nsplit, 64, 512]
   unsigned int* err;
+  long long wait_limit; // bound of every wait, in SM cycles (kWaitLimitCycles unless a test shortens it)
+  int stall;            // test hook: the softmax warps wait on a barrier nothing arrives on
 };
 
 // Raises kernel K's dynamic shared-memory limit once per device (a host-side cost that
@@ -114,6 +121,8 @@ cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* blo
                            int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,
                            cudaStream_t stream, int* launches);
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
+// The fp8-cache decode kernel alone (launch_mla dispatches to it and adds the combine).
+cudaError_t launch_mla_fp8(const MlaArgs& a, cudaStream_t stream);
 int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
 }  // namespace dsa

@@ -67,39 +67,8 @@ static_assert(kIdxListCap % kMlaTile == 0, "list capacity");
 static_assert(kMlaSmem <= 232448, "shared memory");
 static_assert(kLoadThreads * kBatchPieces == kMlaTile * 36, "an fp8 tile is one batch");
 
-// bar.red over named barrier `id` of `count` threads: OR / AND of a predicate.
-__device__ __forceinline__ int bar_or(int id, int count, int v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.or.pred q, %1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return static_cast<int>(r);
-}
-__device__ __forceinline__ int bar_and(int id, int count, int v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbar.red.and.pred q, %1, %2, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return static_cast<int>(r);
-}
-
 __device__ __forceinline__ uint32_t swz(int row, int unit) {  // 128-byte swizzle inside an 8-row atom
   return static_cast<uint32_t>(row * 128 + ((unit ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ int float_exponent(float s) {  // floor(log2 s) for positive normal s
-  return static_cast<int>((__float_as_uint(s) >> 23) & 0xFF) - 127;
-}
-
-__device__ __forceinline__ float exp2i(int e) {  // exact 2^e, clamped to the normal fp32 range
-  e = e < -126 ? -126 : (e > 127 ? 127 : e);
-  return __uint_as_float(static_cast<uint32_t>(e + 127) << 23);
 }
 
 // Per-key tables of one tile buffer, written by the loaders (row j of the tile):
@@ -116,12 +85,6 @@ struct KVMeta {
   int32_t emax[2];
 };
 static_assert(sizeof(KVMeta) <= 1152, "tile table size");
-
-__device__ __forceinline__ float ex2_ftz(float x) {  // hardware 2^x; tiny results flush to zero
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // Read-only global loads that write their destination only when `pred` holds (it keeps
 // the value it had otherwise), so that nothing after the load has to wait for it to
@@ -427,9 +390,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const float oscale = exp2i(e_ref == kNoExp ? 0 : e_ref);
         sOutScale[h] = split_out ? oscale : (l > 0.0f ? oscale / l : 0.0f);
         if (split_out) {
-          float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * 2;
+          float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kPartStats;
           ml[0] = l > 0.0f ? m_run : -INFINITY;
-          ml[1] = l;
+#pragma unroll
+          for (int i = 1; i < kPartStats; ++i) ml[i] = l;   // every value group shares l here
         } else if (a.lse != nullptr) {
           a.lse[static_cast<int64_t>(q) * kHeads + h] =
               l > 0.0f ? (m_run + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -463,6 +427,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
           }
         }
       }
+    }
+    if (!good && a.nsplit > 1 && is_sm) {
+      // an empty partial, so the combine skips this split instead of reading stale data
+      float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kPartStats;
+      ml[0] = -INFINITY;
+#pragma unroll
+      for (int i = 1; i < kPartStats; ++i) ml[i] = 0.0f;
     }
     if (!good && lane == 0) {
       record_error(a.err, DSA_ERR_TIMEOUT, 13);
@@ -685,9 +656,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     if (tid < kHeads) {
       if (split_out) {
-        float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + tid) * 2;
+        float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + tid) * kPartStats;
         ml[0] = -INFINITY;
-        ml[1] = 0.0f;
+#pragma unroll
+        for (int i = 1; i < kPartStats; ++i) ml[i] = 0.0f;
       } else if (a.lse != nullptr) {
         a.lse[static_cast<int64_t>(q) * kHeads + tid] = -INFINITY;
       }
@@ -701,32 +673,39 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 }
 
 // Log-sum-exp merge of the split partials: M = max_s m_s, a_s = 2^(m_s - M),
-// out = sum_s a_s o_s / sum_s a_s l_s, lse = (M + log2 sum_s a_s l_s) * ln 2.
+// out[:, group g] = sum_s a_s o_s / sum_s a_s L_{g,s}, lse = (M + log2 sum_s a_s l_s) * ln 2.
+// L_{g,s} is split s's normaliser for value group g (columns [128 g, 128 g + 128)): its sum
+// of p for a bf16 cache, and for an fp8 cache the sum of the weights its tensor-core PV
+// actually applied to that group, so that each group is normalised by the weights it used.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   pdl_trigger();
   pdl_wait();   // the partials come from the decode kernel
   const int q = blockIdx.x;
   const int h = blockIdx.y;
   const int S = a.nsplit;
-  const float* ml = a.part_ml + static_cast<int64_t>(q) * S * kHeads * 2;
+  const float* ml = a.part_ml + static_cast<int64_t>(q) * S * kHeads * kPartStats;
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(s * kHeads + h) * 2]);
+  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(s * kHeads + h) * kPartStats]);
   float Lsum = 0.0f;
+  float Lg[4] = {0.f, 0.f, 0.f, 0.f};
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   for (int s = 0; s < S; ++s) {
-    const float m = ml[(s * kHeads + h) * 2];
+    const float* st = ml + (s * kHeads + h) * kPartStats;
+    const float m = st[0];
     if (m == -INFINITY) continue;
     const float w = exp2f(m - M);
-    Lsum += w * ml[(s * kHeads + h) * 2 + 1];
+    Lsum += w * st[1];
     const float* o = a.part_o + ((static_cast<int64_t>(q) * S + s) * kHeads + h) * kDimV;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] += w * o[threadIdx.x + 128 * i];
+    for (int i = 0; i < 4; ++i) {
+      Lg[i] += w * st[2 + i];
+      acc[i] += w * o[threadIdx.x + 128 * i];
+    }
   }
-  const float inv = Lsum > 0.0f ? 1.0f / Lsum : 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t off = (static_cast<int64_t>(q) * kHeads + h) * kDimV + threadIdx.x + 128 * i;
-    const float o = acc[i] * inv;
+    const float o = Lg[i] > 0.0f ? acc[i] / Lg[i] : 0.0f;
     if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
     else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
   }
@@ -742,7 +721,8 @@ static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStr
 }
 
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
-  cudaError_t e = fp8 ? launch_mla_t<true>(tmap_q, a, stream) : launch_mla_t<false>(tmap_q, a, stream);
+  // fp8 caches take the e4m3 tensor-core kernel (mla_fp8.cu); bf16 caches this one
+  cudaError_t e = fp8 ? launch_mla_fp8(a, stream) : launch_mla_t<false>(tmap_q, a, stream);
   ++*launches;
   if (e != cudaSuccess || a.nsplit == 1) return e;
   ++*launches;

@@ -281,6 +281,54 @@ def generate(s: CaseSpec) -> dict:
     )
 
 
+def rising_selection(case: dict, tiles: int, climb: float, seed: int = 0, noise_std: float = 0.25):
+    """A selection of `tiles` x 64 latent rows per query whose attention logits climb from
+    one 64-row tile to the next, for tests of the online-softmax rescaling.
+
+    Row h (0..63) of tile t is aimed at head h: noise_std * N(0,1) + t * c_h * q_h / |q_h|,
+    where q_h = q_mla[q, h] and c_h is chosen so that the aimed part adds `climb` log2
+    units to head h's logit per tile (softmax_scale * c_h * |q_h| * log2(e) = climb). So
+    every head's tile maximum rises by about `climb` per tile while the rows keep the
+    generator's magnitude (about 0.5 per element for a few tiles). Rows are stored back in
+    the case's own format (bf16, or E4M3 codes with one amax/448 scale per 128-column group
+    and one for the rope columns), so later tiles also carry larger fp8 scales. Each query
+    uses distinct visible tokens of its own sequence (decode cases, n_q = 1).
+
+    Returns (case copy with the rewritten rows, physical slots [Bq, tiles*64] int32)."""
+    if case["n_q"] != 1:
+        raise ValueError("decode cases only")
+    c = dict(case)
+    c["kv_cache"] = case["kv_cache"].copy()
+    if case["kv_scale"] is not None:
+        c["kv_scale"] = case["kv_scale"].copy()
+    n = tiles * PAGE
+    rng = _rng(seed, 31)
+    k_per_unit = case["softmax_scale"] * math.log2(math.e)
+    phys = np.full((case["Bq"], n), -1, dtype=np.int32)
+    for q in range(case["Bq"]):
+        L = int(case["seq_lens"][q])
+        if L < n:
+            raise ValueError("sequence shorter than the selection")
+        tok = rng.choice(L, size=n, replace=False)
+        slots = case["block_table"][q, tok // PAGE].astype(np.int64) * PAGE + tok % PAGE
+        phys[q] = slots
+        qf = (case["q_mla"][q].astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+        norm = np.linalg.norm(qf, axis=1)                                   # [64]
+        aim = qf / norm[:, None] * (climb / (k_per_unit * norm))[:, None]   # [64, 576]
+        t_of_row = np.arange(n) // PAGE
+        rows = (rng.standard_normal((n, DK)) * noise_std + t_of_row[:, None] * np.tile(aim, (tiles, 1)))
+        rows = rows.astype(np.float32)
+        if case["kv_dtype"] == "bf16":
+            c["kv_cache"][slots] = to_bf16_bits(rows)
+        else:
+            for g in range(KV_GROUPS):
+                lo, hi = g * 128, min(DK, g * 128 + 128)
+                codes, sc = quantize_rows_e4m3(rows[:, lo:hi])
+                c["kv_cache"][slots, lo:hi] = codes
+                c["kv_scale"][slots, g] = sc
+    return c, phys
+
+
 def vis_lengths(case: dict) -> np.ndarray:
     """Visible prefix length of every query: q_pos+1 when causal, else the sequence length.
 

@@ -222,6 +222,21 @@ const char* dsa_status_string(dsa_status status);
  * issued (for launch accounting). */
 int32_t dsa_last_launch_count(void);
 
+/*
+ * Test hook for the bounded waits of the fp8-cache MLA decode kernel (the kernel
+ * mla_sparse_decode, mla_sparse_decode_noalloc and dsa_decode_layer run for an fp8 latent
+ * cache). It applies to the later calls made on this host thread.
+ *  wait_limit_cycles  bound of every wait in SM clock cycles; 0 restores the default
+ *                     (4e9 cycles). Draining in-flight copies and MMAs on the way out
+ *                     always uses the default bound.
+ *  stall              1: the softmax warps wait on a barrier that nothing arrives on, so
+ *                     that wait runs out after wait_limit_cycles; the kernel then stops
+ *                     every role, drains its copies and MMAs, frees its tensor memory,
+ *                     writes empty split partials and records DSA_ERR_TIMEOUT. 0: normal.
+ * Returns DSA_ERR_INVALID_ARG for a negative limit or a stall value other than 0 or 1.
+ */
+dsa_status dsa_test_set_wait_hooks(int64_t wait_limit_cycles, int32_t stall);
+
 #ifdef __cplusplus
 }
 #endif

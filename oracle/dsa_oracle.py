@@ -20,7 +20,8 @@ Every stored code is decoded exactly to fp64 (own E4M3 and bf16 decoders, from t
 OCP 8-bit floating point definition and the bfloat16 bit layout) and multiplied by
 its fp32 scale; all arithmetic after that is fp64.
 
-Readings of points the pages leave open (each one is listed in the design notes):
+Readings of points the pages leave open (the pages name the kernels but give no formula,
+format, page size or tie rule; these are the plainest readings the rest supports):
   * the indexer has no extra 1/sqrt(d) factor, ReLU comes before the head weights;
   * fp8 indexer queries carry one fp32 scale per (query, head); fp8 indexer keys one
     fp32 scale per token; fp8 latent rows five fp32 scales, one per 128-column group of

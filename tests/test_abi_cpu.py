@@ -120,3 +120,10 @@ def test_noalloc_argument_errors():
     assert call(top_k=16385) == dsa.DSA_ERR_INVALID_ARG
     assert call(scale=0.0) == dsa.DSA_ERR_INVALID_ARG
     assert call(status=ctypes.c_void_p(0x100004)) == dsa.DSA_ERR_INVALID_ARG   # status words need 8-byte alignment
+
+
+def test_wait_hook_argument_errors():
+    assert _lib.dsa_test_set_wait_hooks(-1, 0) == dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_test_set_wait_hooks(0, 2) == dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_test_set_wait_hooks(1000, 1) == dsa.DSA_OK
+    assert _lib.dsa_test_set_wait_hooks(0, 0) == dsa.DSA_OK

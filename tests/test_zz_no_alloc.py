@@ -1,12 +1,13 @@
-"""mla_sparse_decode_noalloc against mla_sparse_decode, through the C ABI.
+"""mla_sparse_decode_noalloc against mla_sparse_decode and the fp64 oracle, through the C ABI.
 
 The no-allocation entry point serves callers that cannot allocate device memory (a
 plugin inside an engine that owns all of the GPU's memory, or a loop that must not call
 cudaMalloc/cudaFree): its split partials live in an array the library defines in device
 memory, shared by every call on a device. These tests run two different calls in a row,
 so the second one starts on the scratch contents the first left behind, and compare each
-with the workspace entry point on the same inputs. This file sorts last so that a
-stop-at-first-failure run has finished every other test before it.
+with the workspace entry point on the same inputs and with the oracle's attention on the
+same selection. This file sorts last so that a stop-at-first-failure run has finished
+every other test before it.
 """
 import numpy as np
 import pytest
@@ -77,6 +78,8 @@ def test_noalloc_matches_workspace_entry_on_consecutive_calls():
         ref_out, ref_lse, ref_err = _run(dsa, t, case, physical, noalloc=False)
         assert ref_err == dsa.DSA_OK
         check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"])
+        o_out, o_lse = oracle.mla_sparse_attention(case, physical.cpu().numpy().astype(np.int64))
+        check_attention(out, lse, o_out, o_lse, case["kv_dtype"])
 
 
 def test_noalloc_reports_device_errors_through_status():
