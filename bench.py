@@ -157,7 +157,6 @@ KERNEL_SOURCES = {
     "indexer": ["deepseek_sparse_attention_head_b200/csrc/indexer.cu",
                 "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
     "mla": ["deepseek_sparse_attention_head_b200/csrc/mla.cu",
-            "deepseek_sparse_attention_head_b200/csrc/mla_fp8.cu",
             "deepseek_sparse_attention_head_b200/csrc/common.cuh"],
 }
 
@@ -451,7 +450,7 @@ def run_ours(args, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": (f"{'bf16' if case['idx_dtype'] == 'bf16' else 'e4m3'} indexer + "
-                  f"{'bf16' if case['kv_dtype'] == 'bf16' else 'e4m3 (two-term queries and weights)'} MLA "
+                  f"{'bf16' if case['kv_dtype'] == 'bf16' else 'f16 (e4m3 codes times fp16 row multipliers)'} MLA "
                   f"operands, fp32 accumulate"),
         "data": "synthetic (seeded; dsa_inputs)",
         "config": {

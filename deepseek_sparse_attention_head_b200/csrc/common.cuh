@@ -77,14 +77,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Single-thread bounded wait. Returns false when `limit` SM cycles ran out or another
-// role raised `abort_flag`; the caller then records DSA_ERR_TIMEOUT and unwinds.
+// role raised `abort_flag`; the caller then records DSA_ERR_TIMEOUT and unwinds. With
+// `backoff_ns` > 0 the thread sleeps that long between polls: roles off the critical path
+// then leave issue slots and shared-memory bandwidth to the warps that are.
 __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                         long long limit = kWaitLimitCycles) {
+                                         long long limit = kWaitLimitCycles, unsigned backoff_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
+    if (backoff_ns) __nanosleep(backoff_ns);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
+    if ((i & 255u) == 0u || backoff_ns) {
       if (*abort_flag) return false;
       if (clock64() - t0 > limit) return false;
     }
@@ -95,20 +98,20 @@ __device__ __forceinline__ bool wait_one(uint64_t* bar, uint32_t parity, volatil
 // already completed, the common case); otherwise lane 0 polls alone and the other lanes
 // confirm afterwards, so a waiting warp issues few barrier operations.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          long long limit = kWaitLimitCycles) {
+                                          long long limit = kWaitLimitCycles, unsigned backoff_ns = 0) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, abort_flag, limit);
+  if ((threadIdx.x & 31) == 0) ok = wait_one(bar, parity, abort_flag, limit, backoff_ns);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok) ok = wait_one(bar, parity, abort_flag, limit);
   return __all_sync(0xffffffffu, ok);
 }
 
 // Bounded wait without the abort check, for draining in-flight copies on the way out.
-__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) break;
+    if (clock64() - t0 > limit) break;
   }
 }
 

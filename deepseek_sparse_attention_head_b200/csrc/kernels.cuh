@@ -121,8 +121,6 @@ cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* blo
                            int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,
                            cudaStream_t stream, int* launches);
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
-// The fp8-cache decode kernel alone (launch_mla dispatches to it and adds the combine).
-cudaError_t launch_mla_fp8(const MlaArgs& a, cudaStream_t stream);
 int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
 }  // namespace dsa

@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   uint64_t* p_full = bars + 8;        // [2]
   uint64_t* pv_done = bars + 10;      // [2]
   uint64_t* drain = bars + 12;
+  uint64_t* never = bars + 13;        // test hook only: nothing ever arrives on it
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
   if (ntiles > 0 && warp < 4) {
     // ---------------------------------------------------------------- Q rescale, softmax, epilogue
-    bool good = wait_warp(q_full, 0, abort_flag);
+    bool good = wait_warp(q_full, 0, abort_flag, a.wait_limit);
     const bool q_landed = good;
     {
       const int h = tid >> 1, part = tid & 1;   // 2 threads per head, 36 of its 72 16-byte units each
@@ -244,6 +246,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
+    if (a.stall) {
+      // test hook: a wait that nothing satisfies; it runs out after a.wait_limit cycles
+      good = wait_warp(never, 0, abort_flag, a.wait_limit) && good;
+    }
     good = bar_and(1, 128, good) != 0;
 
     // M=64 puts head h in TMEM lane 32 (h / 16) + h % 16: lanes 0..15 of warp w hold heads
@@ -262,8 +268,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       float y[32];
       int need = 0;
       {
-        const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag) &&
-                         wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag);
+        const bool got = wait_warp(&s_full[b], (T >> 1) & 1, abort_flag, a.wait_limit) &&
+                         wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag, a.wait_limit);
         if (got) {
           tc_fence_after();
           tmem_ld32(tmem + lane_base + b * kMlaTile + 32, y);
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       if (!good) break;
       if (need) {
         // rescale the O^T columns (heads) by alpha; PV(T-1) must have finished first
-        const bool got = wait_warp(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag);
+        const bool got = wait_warp(&pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.wait_limit);
         if (got) {
           tc_fence_after();
 #pragma unroll 1
@@ -400,7 +406,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
       const int last = ntiles - 1;
-      const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag);
+      const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag, a.wait_limit);
       good = bar_and(1, 128, got) != 0;
       if (good) {
         tc_fence_after();
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       record_error(a.err, DSA_ERR_TIMEOUT, 13);
       *abort_flag = 1;
     }
-    if (!q_landed && tid == 0) wait_drain(q_full, 0);   // the Q copy may still be landing
+    if (!q_landed && tid == 0) wait_drain(q_full, 0, a.wait_limit);   // the Q copy may still be landing
     __syncwarp();
   } else if (ntiles > 0 && warp == kMmaWarp) {
     // ---------------------------------------------------------------- tcgen05 issuer (whole warp)
@@ -451,11 +457,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const uint64_t kv_desc0 = sdesc_sw128(smem_u32(sKV), 16, 1024);                 // K-major view
     const uint64_t v_desc0 = sdesc_sw128(smem_u32(sKV), kKVChunk, 1024);            // MN-major view
     const uint64_t p_desc0 = sdesc_sw128(smem_u32(sKV + kPChunk * kKVChunk), 16, 1024);
-    bool good = wait_warp(q_ready, 0, abort_flag);
+    bool good = wait_warp(q_ready, 0, abort_flag, a.wait_limit);
     tc_fence_after();
     auto issue_pv = [&](int T) {
       const int b = T & 1;
-      if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag)) return false;
+      if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag, a.wait_limit)) return false;
       tc_fence_after();
       const uint64_t vb = v_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
       const uint64_t pb = p_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
@@ -473,8 +479,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     };
     for (int T = 0; T < ntiles && good; ++T) {
       const int b = T & 1;
-      if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag)) { good = false; break; }
-      if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag)) { good = false; break; }
+      if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag, a.wait_limit)) { good = false; break; }
+      if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag, a.wait_limit)) { good = false; break; }
       tc_fence_after();
       const uint64_t kb = kv_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
       if (elect_one()) {
@@ -577,7 +583,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     auto step = [&](uint4 (&raw)[kBatchPieces], float (&sc)[kKvGroups], int& my_slot, int T) -> bool {
       const int b = T & 1;
       // the buffer was last read by PV(T-2)
-      const bool ok = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag);
+      const bool ok = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag, a.wait_limit);
       uint32_t* mult = sGrpMeta + b * (kGrpMetaBytes / 4);
       KVMeta* km = sKVMeta + b;
       if (ok && lt < kMlaTile) {
@@ -721,8 +727,7 @@ static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStr
 }
 
 cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
-  // fp8 caches take the e4m3 tensor-core kernel (mla_fp8.cu); bf16 caches this one
-  cudaError_t e = fp8 ? launch_mla_fp8(a, stream) : launch_mla_t<false>(tmap_q, a, stream);
+  cudaError_t e = fp8 ? launch_mla_t<true>(tmap_q, a, stream) : launch_mla_t<false>(tmap_q, a, stream);
   ++*launches;
   if (e != cudaSuccess || a.nsplit == 1) return e;
   ++*launches;

@@ -261,11 +261,28 @@ __device__ __forceinline__ void gather_load(const float* row, int base, int hi_s
 }
 
 // Bit 4 j + t set when key t of cur[j] (index base + 4 (j * 1024 + tid) + t) is below
-// hi_s (checked unless kWhole) and at least thr.
+// hi_s (checked unless kWhole) and at least thr. When thr is the key of a non-negative
+// float (thr >= 0x80000000), key >= thr holds exactly when the score's bit pattern, read
+// as a signed integer, is at least thr's float bit pattern: negative scores (and negative
+// NaNs) are negative integers, and non-negative ones (+inf and +NaN included) order like
+// their keys. One integer compare per score instead of the key transform.
 template <bool kWhole>
 __device__ __forceinline__ uint32_t gather_takes(const float4 (&cur)[kGatherU / 4], int base, int hi_s,
                                                  uint32_t thr) {
   uint32_t takes = 0;
+  if (thr >= 0x80000000u) {
+    const int tb = static_cast<int>(thr & 0x7FFFFFFFu);
+#pragma unroll
+    for (int j = 0; j < kGatherU / 4; ++j) {
+      const int s_ = base + 4 * (j * kTopkThreads + static_cast<int>(threadIdx.x));
+      const int e[4] = {__float_as_int(cur[j].x), __float_as_int(cur[j].y), __float_as_int(cur[j].z),
+                        __float_as_int(cur[j].w)};
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if ((kWhole || s_ + t < hi_s) && e[t] >= tb) takes |= 1u << (4 * j + t);
+    }
+    return takes;
+  }
 #pragma unroll
   for (int j = 0; j < kGatherU / 4; ++j) {
     const int s_ = base + 4 * (j * kTopkThreads + static_cast<int>(threadIdx.x));
@@ -291,25 +308,25 @@ __device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr,
   float4 nxt[kGatherU / 4];
   for (int base = lo_s; base < hi_s; base += kGatherBatch) {
     if (base + kGatherBatch < hi_s) gather_load(row, base + kGatherBatch, hi_s, nxt);
-    const uint32_t takes = base + kGatherBatch <= hi_s ? gather_takes<true>(cur, base, hi_s, thr)
-                                                        : gather_takes<false>(cur, base, hi_s, thr);
+    uint32_t takes = base + kGatherBatch <= hi_s ? gather_takes<true>(cur, base, hi_s, thr)
+                                                  : gather_takes<false>(cur, base, hi_s, thr);
     uint32_t c = warp_reserve(counter, static_cast<uint32_t>(__popc(takes)));
+    // only the taken keys (a few percent) are visited
+    while (takes != 0u) {
+      const int bit = __ffs(takes) - 1;
+      takes &= takes - 1u;
+      const int j = bit >> 2, t = bit & 3;
+      float e = cur[0].x;
 #pragma unroll
-    for (int j = 0; j < kGatherU / 4; ++j) {
-      const int s_ = base + 4 * (j * kTopkThreads + tid);
-      const float e[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        if (takes & (1u << (4 * j + t))) {
-          const uint32_t u = order_key(e[t]);
-          if (c < cap) {
-            out_key[c] = u;
-            out_idx[c] = s_ + t;
-          }
-          ++c;
-          lmax = max(lmax, u - thr);
-        }
+      for (int jj = 0; jj < kGatherU / 4; ++jj)
+        if (jj == j) e = t == 0 ? cur[jj].x : (t == 1 ? cur[jj].y : (t == 2 ? cur[jj].z : cur[jj].w));
+      const uint32_t u = order_key(e);
+      if (c < cap) {
+        out_key[c] = u;
+        out_idx[c] = base + 4 * (j * kTopkThreads + tid) + t;
       }
+      ++c;
+      lmax = max(lmax, u - thr);
     }
 #pragma unroll
     for (int j = 0; j < kGatherU / 4; ++j) cur[j] = nxt[j];

@@ -21,7 +21,7 @@ import pytest
 
 import oracle
 from dsa_inputs import CaseSpec, generate, rising_selection
-from tests.compare import check_attention
+from tests.compare import check_attention, fp8_lse_bound
 
 TILE = 64
 LOG2E = 1.0 / math.log(2.0)
@@ -86,7 +86,8 @@ def test_mla_matches_oracle_on_rising_logits(name):
     out, lse, err = GpuCase(case).mla(phys)
     assert err == 0
     ref_out, ref_lse = oracle.mla_sparse_attention(case, phys.astype(np.int64))
-    check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"])
+    bound = fp8_lse_bound(case, phys) if case["kv_dtype"] == "fp8" else None
+    check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"], lse_bound=bound)
 
 
 @pytest.mark.gpu
@@ -100,4 +101,5 @@ def test_mla_matches_oracle_on_falling_logits(name):
     out, lse, err = GpuCase(case).mla(rev)
     assert err == 0
     ref_out, ref_lse = oracle.mla_sparse_attention(case, rev.astype(np.int64))
-    check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"])
+    bound = fp8_lse_bound(case, rev) if case["kv_dtype"] == "fp8" else None
+    check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"], lse_bound=bound)
