@@ -88,9 +88,10 @@ static_assert(sizeof(KVMeta) <= 1152, "tile table size");
 
 // Read-only global loads that write their destination only when `pred` holds (it keeps
 // the value it had otherwise), so that nothing after the load has to wait for it to
-// choose between the loaded value and a default.
+// choose between the loaded value and a default. The gathered rows are used once: they do
+// not allocate in L1, which is small next to this kernel's shared memory.
 __device__ __forceinline__ void ldg_pred(uint4& v, const void* p, bool pred) {
-  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}\n"
+  asm("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %5, 0;\n\t@q ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}\n"
       : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
       : "l"(p), "r"(static_cast<uint32_t>(pred)));
 }
@@ -207,6 +208,36 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   // fp16 operands for an fp8 cache, bf16 for a bf16 cache
   const uint32_t fmt = FP8 ? 0u : 1u;
 
+  // Output epilogue, shared by the softmax warps and the loaders once O is final: warp w
+  // reads TMEM lanes 32 (w % 4) .. + 31 (value dims), and the three warps of a lane quadrant
+  // (r = 0, 1, 2) take every third of its eight 32-head column blocks.
+  auto write_out = [&](int r) {
+    const bool split_out = a.nsplit > 1;
+    const int quad = warp & 3;
+    const uint32_t lb = static_cast<uint32_t>(quad * 32) << 16;
+    tc_fence_after();
+#pragma unroll 1
+    for (int k = r; k < 8; k += 3) {
+      const int d = k >> 1, half = k & 1;
+      const int dim = d * 128 + quad * 32 + lane;
+      float v[32];
+      tmem_ld32(tmem + kTmemO + lb + d * 64 + half * 32, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int hh = half * 32 + i;
+        const float o = v[i] * sOutScale[hh];
+        if (split_out) {
+          a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = o;
+        } else {
+          const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
+          if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
+          else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
+        }
+      }
+    }
+  };
+  constexpr int kEpiBar = 3, kEpiThreads = 4 * 32 + kLoadThreads;   // softmax warps + loaders
+
   if (ntiles > 0 && warp < 4) {
     // ---------------------------------------------------------------- Q rescale, softmax, epilogue
     bool good = wait_warp(q_full, 0, abort_flag, a.wait_limit);
@@ -253,8 +284,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     good = bar_and(1, 128, good) != 0;
 
     // M=64 puts head h in TMEM lane 32 (h / 16) + h % 16: lanes 0..15 of warp w hold heads
-    // 16w .. 16w+15. Lane l < 16 takes keys 0..31 of its head, lane l + 16 keys 32..63 of
-    // the same head (handed over by shuffle); both keep identical running statistics.
+    // 16w .. 16w+15. Lane l < 16 reads keys 0..31 of its head, lane l + 16 keys 32..63 of
+    // the same head (one two-range TMEM load); both keep identical running statistics.
     const bool is_sm = lane < 16;           // the lane that writes per-head state
     const int h = warp * 16 + (lane & 15);
     const int jb = lane < 16 ? 0 : 32;      // this lane's keys: jb .. jb+31
@@ -272,17 +303,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                          wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag, a.wait_limit);
         if (got) {
           tc_fence_after();
-          tmem_ld32(tmem + lane_base + b * kMlaTile + 32, y);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __shfl_sync(0xffffffffu, y[i], lane & 15);
-          {
-            float y0[32];
-            tmem_ld32(tmem + lane_base + b * kMlaTile, y0);
-            if (is_sm) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) y[i] = y0[i];
-            }
-          }
+          tmem_ld_16x32bx2_x32(tmem + lane_base + b * kMlaTile, y);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&s_empty[b]);
@@ -388,7 +409,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     // the two lanes of a head hold halves of its normaliser
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
-    // ---- epilogue: warps 0..3 read O^T (lanes = dims), softmax threads supply per-head scales
+    // ---- epilogue: per-head scales and statistics, then O^T out of TMEM with the loaders
+    bool got = false;
     if (good) {
       const bool split_out = a.nsplit > 1;
       if (is_sm) {
@@ -406,34 +428,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       }
       const int last = ntiles - 1;
-      const bool got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag, a.wait_limit);
-      good = bar_and(1, 128, got) != 0;
-      if (good) {
-        tc_fence_after();
-        const int dim_in_tile = warp * 32 + lane;
-#pragma unroll 1
-        for (int d = 0; d < 4; ++d) {
-          const int dim = d * 128 + dim_in_tile;
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            float v[32];
-            tmem_ld32(tmem + kTmemO + lane_base + d * 64 + half * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int hh = half * 32 + i;
-              const float o = v[i] * sOutScale[hh];
-              if (split_out) {
-                a.part_o[((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + hh) * kDimV + dim] = o;
-              } else {
-                const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
-                if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
-                else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
-              }
-            }
-          }
-        }
-      }
+      got = wait_warp(&pv_done[last & 1], (last >> 1) & 1, abort_flag, a.wait_limit);
     }
+    // a failure stops the other roles now, not after the loaders' next wait runs out
+    if (!(good && got) && lane == 0) *abort_flag = 1;
+    // O is final and the scales are published: the loaders join the readout
+    good = bar_and(kEpiBar, kEpiThreads, good && got) != 0;
+    if (good) write_out(0);
     if (!good && a.nsplit > 1 && is_sm) {
       // an empty partial, so the combine skips this split instead of reading stale data
       float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kPartStats;
@@ -461,7 +462,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     tc_fence_after();
     auto issue_pv = [&](int T) {
       const int b = T & 1;
-      if (!wait_warp(&p_full[b], (T >> 1) & 1, abort_flag, a.wait_limit)) return false;
       tc_fence_after();
       const uint64_t vb = v_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
       const uint64_t pb = p_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
@@ -475,12 +475,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tc_commit(&pv_done[b]);
       }
       __syncwarp();
-      return true;
     };
-    for (int T = 0; T < ntiles && good; ++T) {
+    auto issue_qk = [&](int T) {
       const int b = T & 1;
-      if (!wait_warp(&kv_full[b], (T >> 1) & 1, abort_flag, a.wait_limit)) { good = false; break; }
-      if (!wait_warp(&s_empty[b], ((T >> 1) & 1) ^ 1, abort_flag, a.wait_limit)) { good = false; break; }
       tc_fence_after();
       const uint64_t kb = kv_desc0 + static_cast<uint64_t>((b * kKVBytes) >> 4);
       if (elect_one()) {
@@ -493,9 +490,26 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         tc_commit(&s_full[b]);
       }
       __syncwarp();
-      if ((T & 1) && !(issue_pv(T - 1) && issue_pv(T))) { good = false; break; }
+    };
+    // Whichever is ready first: QK of the next tile (its buffer converted, its S slot read
+    // by the softmax) or PV of the oldest tile whose weights are written. PV(T) then follows
+    // the softmax at once instead of waiting for tile T + 1's conversion, and the loaders,
+    // who refill a buffer after its PV, start sooner.
+    int nq = 0, np = 0;   // next QK tile, next PV tile (np <= nq)
+    long long t_idle = clock64();
+    for (uint32_t spin = 0; good && np < ntiles;) {
+      if (nq < ntiles && __all_sync(0xffffffffu, mbar_test_wait(&kv_full[nq & 1], (nq >> 1) & 1) &&
+                                                     mbar_test_wait(&s_empty[nq & 1], ((nq >> 1) & 1) ^ 1))) {
+        issue_qk(nq++);
+      } else if (np < nq && __all_sync(0xffffffffu, mbar_test_wait(&p_full[np & 1], (np >> 1) & 1))) {
+        issue_pv(np++);
+      } else {
+        if ((++spin & 255u) == 0u && (*abort_flag || clock64() - t_idle > a.wait_limit)) good = false;
+        continue;
+      }
+      spin = 0;
+      t_idle = clock64();
     }
-    if (good && (ntiles & 1) && !issue_pv(ntiles - 1)) good = false;
     if (!good && lane == 0) {
       record_error(a.err, DSA_ERR_TIMEOUT, 10);
       *abort_flag = 1;
@@ -645,6 +659,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       *abort_flag = 1;
     }
     __syncwarp();
+    // the output epilogue with the softmax warps (they publish the per-head scales first)
+    if (bar_and(kEpiBar, kEpiThreads, good) != 0) write_out(warp <= kLoadWarp0 + 3 ? 1 : 2);
   }
 
   if (ntiles == 0) {
