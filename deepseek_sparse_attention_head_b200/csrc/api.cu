@@ -3,6 +3,7 @@
 // synchronisation except in dsa_get_error.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <mutex>
@@ -78,17 +79,35 @@ dsa_status check_paging(const dsa_paging* pg) {
   return DSA_OK;
 }
 
-int mla_splits_for(int Bq, int top_k, int* keys_per_split) {
-  const int sms = device_sms();
+// KV splits of the MLA decode for Bq queries of top_k keys. The count minimises an
+// estimate of the time, (waves of CTAs over the SMs) x (tiles per CTA + the CTA's fixed
+// cost in tiles, + one for the combine when split), over counts that keep Bq x splits
+// within max_ctas (the caller's budget for partial buffers; 0: four waves). One CTA per SM.
+int mla_splits_for(int Bq, int top_k, int* keys_per_split, int max_ctas = 0) {
+  constexpr int kFixedTiles = 4;   // prologue + epilogue, about four 64-key tiles
+  const int sms = device_sms() > 0 ? device_sms() : 1;
   const int tile = mla_tile_keys();
   const int ntiles = (top_k + tile - 1) / tile;
-  int s = sms > 0 ? sms / (Bq > 0 ? Bq : 1) : 1;
-  if (s < 1) s = 1;
-  if (s > ntiles) s = ntiles;
-  int kps = ((ntiles + s - 1) / s) * tile;
-  s = (top_k + kps - 1) / kps;
+  const int64_t bq = Bq > 0 ? Bq : 1;
+  const int64_t cap = max_ctas > 0 ? std::max<int64_t>(max_ctas, bq) : std::max<int64_t>(4LL * sms, bq);
+  int best_s = 1, best_tiles = ntiles;
+  int64_t best_cost = -1;
+  for (int s = 1; s <= ntiles; ++s) {
+    const int tps = (ntiles + s - 1) / s;           // tiles per split
+    const int se = (ntiles + tps - 1) / tps;        // splits actually used
+    if (se != s) continue;                          // the same layout as a smaller count
+    if (bq * se > cap) break;
+    const int64_t waves = (bq * se + sms - 1) / sms;
+    const int64_t cost = waves * (tps + kFixedTiles + (se > 1 ? 1 : 0));
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_s = se;
+      best_tiles = tps;
+    }
+  }
+  const int kps = best_tiles * tile;
   if (keys_per_split) *keys_per_split = kps;
-  return s;
+  return (top_k + kps - 1) / kps;
 }
 
 struct Layout {
@@ -508,7 +527,8 @@ extern "C" dsa_status mla_sparse_decode_noalloc(int32_t Bq, const void* q, const
   if (s != DSA_OK) return s;
   if (status != nullptr && !aligned(status, 8)) return DSA_ERR_INVALID_ARG;
   int kps = 0;
-  const int nsplit = mla_splits_for(Bq, top_k, &kps);
+  // at most one (query, split) pair per SM, which the static scratch is sized for
+  const int nsplit = mla_splits_for(Bq, top_k, &kps, device_sms());
   const Layout lay = layout_for(0, Bq, 0, top_k, -1, nsplit);
   if (lay.total > kMlaStaticScratchBytes) return DSA_ERR_WORKSPACE;
   uint8_t* scratch = mla_static_scratch();

@@ -53,6 +53,8 @@ class CaseSpec:
     out_dtype: str = "bf16"          # "fp32" | "bf16"
     n_q: int = 1                     # queries per sequence (1 = decode)
     q_pos: Optional[tuple] = None    # causal positions of the n_q queries of a sequence
+    q_tail: bool = False             # no q_pos: each sequence's n_q queries sit at its last
+                                     # n_q positions (speculative multi-token decode)
     n_planted: int = 32              # hot tokens per sequence (decode only)
     planted_mode: str = "uniform"    # "uniform" | "loguniform"
     seed: int = 0
@@ -84,6 +86,9 @@ CONFIGS = {
                      planted_mode="loguniform", seed=3),
     "cfg4": CaseSpec("cfg4", (65536,), top_k=2048, n_q=2048,
                      q_pos=tuple(range(63488, 65536)), n_planted=0, seed=4),
+    # not one of the five graded configs: the serving workload's rows with three queries
+    # each at their last three positions, as a speculative (multi-token) decode verifies them
+    "mtp": CaseSpec("mtp", _cfg2_lens(2), top_k=2048, n_q=3, q_tail=True, n_planted=0, seed=5),
 }
 
 WORKLOAD_NAMES = {
@@ -92,6 +97,7 @@ WORKLOAD_NAMES = {
     "cfg2": "serving-shaped fp8 decode B=64 L~U[2048,65536] top_k=2048",
     "cfg3": "long-context fp8 decode B=1 L=1048576 top_k=2048",
     "cfg4": "chunked-prefill fp8 n_q=2048 at 63488..65535 of L=65536 top_k=2048",
+    "mtp": "speculative decode fp8 B=64 L~U[2048,65536] n_q=3 at each row's last 3 positions top_k=2048",
 }
 
 
@@ -187,6 +193,10 @@ def generate(s: CaseSpec) -> dict:
         if len(s.q_pos) != n_q:
             raise ValueError("q_pos must list n_q positions")
         q_pos = np.tile(np.asarray(s.q_pos, dtype=np.int32), B)
+    elif s.q_tail:
+        if n_q > 1 and int(lens.min(initial=n_q)) < n_q:
+            raise ValueError("q_tail needs every sequence to hold at least n_q tokens")
+        q_pos = (lens[:, None] - n_q + np.arange(n_q)[None, :]).reshape(-1).astype(np.int32)
 
     # ---- indexer queries and head weights
     rq = _rng(s.seed, 2)

@@ -1,5 +1,6 @@
 """The serving-size workloads (B=64 serving decode, one 1M-token stream, 2048-query chunked
-prefill) through the fused decode layer, the call bench.py times.
+prefill, and the serving rows with three speculative queries each) through the fused
+decode layer, the call bench.py times.
 
 The oracle recomputes sampled query rows element by element (scores, top-k set up to
 near-ties, attention on the GPU's own selection). Every row is checked against
@@ -27,6 +28,10 @@ def _sample(name, case):
     if Bq == 1:
         return [0]
     picks = {0, Bq - 1, int(np.argmax(vis)), int(np.argmin(vis))}
+    if case["n_q"] > 1:
+        # every query of the first and of the shortest row (causal visibility differs by one)
+        for b in (0, int(np.argmin(case["seq_lens"]))):
+            picks |= set(range(b * case["n_q"], (b + 1) * case["n_q"]))
     dense = np.nonzero(vis <= case["top_k"])[0]
     if dense.size:
         picks.add(int(dense[0]))
@@ -49,7 +54,7 @@ def _run(name):
     return case, q, sc, serr, layer
 
 
-@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4"])
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4", "mtp"])
 def test_full_size_every_row_properties(name):
     case, _, _, serr, r = _run(name)
     assert serr == 0 and r["err"] == 0
@@ -70,7 +75,7 @@ def test_full_size_every_row_properties(name):
     assert np.all(np.isfinite(r["lse"]) == (vis > 0)[:, None])
 
 
-@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4"])
+@pytest.mark.parametrize("name", ["cfg2", "cfg3", "cfg4", "mtp"])
 def test_full_size_sampled_rows_against_oracle(name):
     case, q, sc, _, r = _run(name)
     vis = oracle.visible_lengths(case)[q]

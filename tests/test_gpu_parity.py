@@ -21,6 +21,12 @@ SMALL = {
     "empty_row": CaseSpec("empty_row", (0, 50, 700), top_k=96, seed=35),
     "many_rows": CaseSpec("many_rows", tuple(range(40, 40 + 37 * 97, 97)), top_k=128, seed=36),
     "wide_table": CaseSpec("wide_table", (500, 1000), top_k=256, max_pages=40, extra_pages=7, seed=37),
+    # speculative decode: every row's last n_q positions are queries (causal, so they see
+    # L - n_q + 1 .. L tokens); one row is shorter than top_k and takes the dense path
+    "mtp_small": CaseSpec("mtp_small", (300, 1000, 70, 2100), top_k=128, n_q=3, q_tail=True, n_planted=0,
+                          seed=38),
+    "mtp_bf16": CaseSpec("mtp_bf16", (129, 640), top_k=64, n_q=4, q_tail=True, idx_dtype="bf16", kv_dtype="bf16",
+                         out_dtype="fp32", n_planted=0, seed=39),
 }
 FULL = ["cfg0", "cfg1"]
 

@@ -131,3 +131,12 @@ def test_algorithmic_bytes_by_hand():
     assert ab["query_side"] == 2 * per_query
     assert ab["total"] == ab["indexer"] + ab["mla"] + ab["query_side"]
     assert dsa_inputs.indexer_flops(case) == 2 * H * DI * 120
+
+
+def test_q_tail_places_queries_at_each_rows_last_positions():
+    c = dsa_inputs.generate(dsa_inputs.CaseSpec("tail", (5, 9, 3), top_k=4, n_q=3, q_tail=True, n_planted=0, seed=9))
+    assert c["q_pos"].tolist() == [2, 3, 4, 6, 7, 8, 0, 1, 2]
+    m = dsa_inputs.spec("mtp")
+    assert m.n_q == 3 and m.q_tail and m.seq_lens == dsa_inputs.spec("cfg2").seq_lens and m.Bq == 192
+    with pytest.raises(ValueError):
+        dsa_inputs.generate(dsa_inputs.CaseSpec("short", (5, 2), top_k=4, n_q=3, q_tail=True, n_planted=0))

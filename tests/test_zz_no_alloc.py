@@ -22,8 +22,8 @@ pytestmark = pytest.mark.gpu
 CASES = [
     # fp8 latent cache, few queries: many KV splits, so the partials are in use
     CaseSpec("noalloc_fp8", (900, 3000, 61), top_k=256, seed=51),
-    # bf16 cache, fp32 output, more queries and a shorter list: another split layout
-    CaseSpec("noalloc_bf16", tuple(range(50, 50 + 29 * 71, 71)), top_k=128, idx_dtype="bf16", kv_dtype="bf16",
+    # bf16 cache, fp32 output, more queries (four splits of two tiles): another split layout
+    CaseSpec("noalloc_bf16", tuple(range(50, 50 + 29 * 71, 71)), top_k=512, idx_dtype="bf16", kv_dtype="bf16",
              out_dtype="fp32", seed=52),
 ]
 
