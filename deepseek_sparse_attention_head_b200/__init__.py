@@ -22,7 +22,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa_b20
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_WORKSPACE, \
     DSA_ERR_DEVICE_BOUNDS, DSA_ERR_TIMEOUT = range(7)
-DSA_BF16, DSA_FP8_E4M3, DSA_FP32 = range(3)
+DSA_BF16, DSA_FP8_E4M3, DSA_FP32, DSA_FP8_E4M3_ROPE_BF16 = range(4)
 DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_PAGEMAP, DSA_OP_LAYER = range(4)
 
 PAGE_SIZE = 64
@@ -94,6 +94,14 @@ def exported_symbols():
 
 
 # ---------------------------------------------------------------------- helpers
+
+def _kv_code(t: torch.Tensor) -> int:
+    """Latent-cache layout code: uint8 rows 656 bytes wide are the packed layout (E4M3 codes,
+    four fp32 scales, bf16 rope); other caches follow their element type."""
+    if t.dtype == torch.uint8 and t.dim() >= 1 and t.shape[-1] == 656:
+        return DSA_FP8_E4M3_ROPE_BF16
+    return _dtype_code(t)
+
 
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
@@ -223,7 +231,7 @@ def dsa_pagemap(paging: Paging, logical: torch.Tensor, physical: torch.Tensor, w
 def mla_sparse_decode(q: torch.Tensor, kv_cache: torch.Tensor, kv_scale, physical: torch.Tensor,
                       softmax_scale: float, out: torch.Tensor, lse, workspace: torch.Tensor, stream=None):
     Bq = int(q.shape[0])
-    st = _lib.mla_sparse_decode(Bq, _ptr(q), _ptr(kv_cache), _dtype_code(kv_cache), _ptr(kv_scale),
+    st = _lib.mla_sparse_decode(Bq, _ptr(q), _ptr(kv_cache), _kv_code(kv_cache), _ptr(kv_scale),
                                 int(kv_cache.shape[0]), _ptr(physical), int(physical.shape[-1]),
                                 float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(lse), _ptr(workspace),
                                 workspace.numel(), _stream(stream))
@@ -238,7 +246,7 @@ def mla_sparse_decode_noalloc(q: torch.Tensor, kv_cache: torch.Tensor, kv_scale,
     For callers that cannot allocate device memory. `status`, if given, is a device int32
     tensor of 2 elements that receives the call's device-side error words."""
     Bq = int(q.shape[0])
-    st = _lib.mla_sparse_decode_noalloc(Bq, _ptr(q), _ptr(kv_cache), _dtype_code(kv_cache), _ptr(kv_scale),
+    st = _lib.mla_sparse_decode_noalloc(Bq, _ptr(q), _ptr(kv_cache), _kv_code(kv_cache), _ptr(kv_scale),
                                         int(kv_cache.shape[0]), _ptr(physical), int(physical.shape[-1]),
                                         float(softmax_scale), _ptr(out), _dtype_code(out), _ptr(lse),
                                         _ptr(status), _stream(stream))
@@ -251,7 +259,7 @@ def dsa_decode_layer(paging: Paging, q_idx, q_scale, head_w, k_cache, k_scale, q
                      logical_out=None, physical_out=None, stream=None):
     """Indexer -> top-k + page map -> MLA sparse decode, one call on one stream."""
     st = _lib.dsa_decode_layer(paging.ref(), _ptr(q_idx), _dtype_code(q_idx), _ptr(q_scale), _ptr(head_w),
-                               _ptr(k_cache), _ptr(k_scale), _ptr(q_mla), _ptr(kv_cache), _dtype_code(kv_cache),
+                               _ptr(k_cache), _ptr(k_scale), _ptr(q_mla), _ptr(kv_cache), _kv_code(kv_cache),
                                _ptr(kv_scale), int(top_k), float(softmax_scale), _ptr(out), _dtype_code(out),
                                _ptr(lse), _ptr(logical_out), _ptr(physical_out), _ptr(workspace),
                                workspace.numel(), _stream(stream))

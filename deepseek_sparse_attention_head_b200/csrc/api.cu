@@ -267,7 +267,8 @@ dsa_status run_mla(int Bq, const void* q, const void* kv, dsa_dtype kv_dtype, co
   a.err = err_word(ws);
   a.wait_limit = g_test_wait_limit > 0 ? g_test_wait_limit : kWaitLimitCycles;
   a.stall = g_test_stall;
-  return cuda_status(launch_mla(kv_dtype == DSA_FP8_E4M3, tq, a, st, &g_launches));
+  const int kvf = kv_dtype == DSA_FP8_E4M3 ? kKvFp8 : kv_dtype == DSA_FP8_E4M3_ROPE_BF16 ? kKvFp8Packed : kKvBf16;
+  return cuda_status(launch_mla(kvf, tq, a, st, &g_launches));
 }
 
 dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -300,8 +301,8 @@ dsa_status check_mla_inputs(int Bq, const void* q, const void* kv, dsa_dtype kv_
   if (!(scale > 0.0f) || !std::isfinite(scale)) return DSA_ERR_INVALID_ARG;
   if (kv_dtype == DSA_FP8_E4M3) {
     if (kv_scale == nullptr) return DSA_ERR_INVALID_ARG;
-  } else if (kv_dtype == DSA_BF16) {
-    if (kv_scale != nullptr) return DSA_ERR_INVALID_ARG;
+  } else if (kv_dtype == DSA_BF16 || kv_dtype == DSA_FP8_E4M3_ROPE_BF16) {
+    if (kv_scale != nullptr) return DSA_ERR_INVALID_ARG;   // no scale plane (packed rows carry theirs)
   } else {
     return DSA_ERR_INVALID_ARG;
   }

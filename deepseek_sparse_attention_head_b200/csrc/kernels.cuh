@@ -120,7 +120,11 @@ cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* lau
 cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,
                            int num_pages, const int32_t* logical, int32_t* physical, unsigned int* err,
                            cudaStream_t stream, int* launches);
-cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
+// Latent cache layouts of the MLA decode: bf16 rows; E4M3 rows with a [rows, 5] fp32 scale
+// plane; packed 656-byte rows (512 E4M3 codes, four fp32 scales, 64 bf16 rope values).
+constexpr int kKvBf16 = 0, kKvFp8 = 1, kKvFp8Packed = 2;
+constexpr int kPackedRowBytes = kDimV + 4 * 4 + 2 * (kDimK - kDimV);
+cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
 int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
 }  // namespace dsa

@@ -101,6 +101,17 @@ __device__ __forceinline__ void ldg_pred(float& v, const float* p, bool pred) {
       : "l"(p), "r"(static_cast<uint32_t>(pred)));
 }
 
+// Packed 656-byte rows, a tile's pieces p in [0, 2560): p < 2048 is code piece p % 32 of row
+// p / 32 (bytes 16 (p % 32)); the rest is rope piece (p - 2048) % 8 of row (p - 2048) / 8
+// (bytes 528 + 16 ((p - 2048) % 8)).
+constexpr int kPackedCodePieces = kMlaTile * 32;
+__device__ __forceinline__ int packed_row(int p) {
+  return p < kPackedCodePieces ? p >> 5 : (p - kPackedCodePieces) >> 3;
+}
+__device__ __forceinline__ int packed_byte(int p) {
+  return p < kPackedCodePieces ? 16 * (p & 31) : kDimV + 16 + 16 * ((p - kPackedCodePieces) & 7);
+}
+
 // Four E4M3 codes -> four fp16 (exact) times the fp16 multiplier pair m2.
 __device__ __forceinline__ void dequant4_f16(uint32_t w, __half2 m2, uint32_t& o0, uint32_t& o1) {
   const __half2_raw r01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
@@ -111,9 +122,13 @@ __device__ __forceinline__ void dequant4_f16(uint32_t w, __half2 m2, uint32_t& o
   o1 = *reinterpret_cast<uint32_t*>(&h23);
 }
 
-template <bool FP8>
+// KVF: the latent cache layout, kKvBf16, kKvFp8 (576 E4M3 codes per row + a [rows, 5] fp32
+// scale plane) or kKvFp8Packed (656-byte rows: 512 codes, four fp32 scales, 64 bf16 rope).
+template <int KVF>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaArgs a) {
+  constexpr bool FP8 = KVF != kKvBf16;            // fp16 operands from E4M3 codes
+  constexpr bool PACKED = KVF == kKvFp8Packed;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
@@ -529,44 +544,75 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // batch of 9 pieces per thread, loaded two tiles ahead; a bf16 tile is two batches, the
     // second loaded when it is needed.
     const int lt = tid - kLoadWarp0 * 32;
-    constexpr int kRowPieces = FP8 ? 36 : 72;
-    constexpr int kRowBytes = FP8 ? kDimK : 2 * kDimK;
+    // Packed rows: a tile's first 2048 pieces are the codes (32 per row, bytes 16 c), the
+    // last 512 the bf16 rope (8 per row, bytes 528 + 16 u, past the four scales); thread t
+    // owns pieces t + 256 i, so its pieces i < 8 are codes and 8, 9 rope, the same in every
+    // lane of a warp.
+    constexpr int kRowPieces = PACKED ? 40 : (FP8 ? 36 : 72);
+    constexpr int kRowBytes = PACKED ? kPackedRowBytes : (FP8 ? kDimK : 2 * kDimK);
     constexpr int kBatches = FP8 ? 1 : 2;
-    uint4 rawA[kBatchPieces], rawB[kBatchPieces];
+    constexpr int kPieces = PACKED ? 10 : kBatchPieces;   // per thread and batch
+    static_assert(kLoadThreads * kPieces * kBatches == kMlaTile * kRowPieces, "a tile is whole batches");
+    uint4 rawA[kPieces], rawB[kPieces];
     float scA[kKvGroups], scB[kKvGroups];
     int slotA = -1, slotB = -1;   // row lt's slot (threads lt < 64)
     // all slot lookups first, then all loads, so that no lookup waits behind a load
-    auto fetch = [&](uint4 (&raw)[kBatchPieces], int T, int batch) {
-      int sl[kBatchPieces];
+    auto fetch = [&](uint4 (&raw)[kPieces], int T, int batch) {
+      int sl[kPieces];
 #pragma unroll
-      for (int i = 0; i < kBatchPieces; ++i) {
-        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
-        sl[i] = slot_at(T, p / kRowPieces);
+      for (int i = 0; i < kPieces; ++i) {
+        const int p = lt + kLoadThreads * (batch * kPieces + i);
+        sl[i] = slot_at(T, PACKED ? packed_row(p) : p / kRowPieces);
       }
 #pragma unroll
-      for (int i = 0; i < kBatchPieces; ++i) {
-        const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
-        const int c16 = p % kRowPieces;
+      for (int i = 0; i < kPieces; ++i) {
+        const int p = lt + kLoadThreads * (batch * kPieces + i);
+        const int byte = PACKED ? packed_byte(p) : (p % kRowPieces) * 16;
         raw[i] = make_uint4(0u, 0u, 0u, 0u);
-        ldg_pred(raw[i], a.kv + static_cast<int64_t>(max(sl[i], 0)) * kRowBytes + c16 * 16, sl[i] >= 0);
+        ldg_pred(raw[i], a.kv + static_cast<int64_t>(max(sl[i], 0)) * kRowBytes + byte, sl[i] >= 0);
       }
     };
     auto fetch_meta = [&](float (&sc)[kKvGroups], int& my_slot, int T) {
       if (lt < kMlaTile) {
         my_slot = slot_at(T, lt);
 #pragma unroll
-        for (int k = 0; k < kKvGroups; ++k) {
-          sc[k] = 0.0f;
-          if (FP8) ldg_pred(sc[k], a.kv_scale + static_cast<int64_t>(max(my_slot, 0)) * kKvGroups + k, my_slot >= 0);
+        for (int k = 0; k < kKvGroups; ++k) sc[k] = 0.0f;
+        if (PACKED) {
+          // the four group scales sit in the row, after its 512 codes; the rope has none
+          uint4 s4 = make_uint4(0u, 0u, 0u, 0u);
+          ldg_pred(s4, a.kv + static_cast<int64_t>(max(my_slot, 0)) * kRowBytes + kDimV, my_slot >= 0);
+          sc[0] = __uint_as_float(s4.x);
+          sc[1] = __uint_as_float(s4.y);
+          sc[2] = __uint_as_float(s4.z);
+          sc[3] = __uint_as_float(s4.w);
+        } else if (FP8) {
+#pragma unroll
+          for (int k = 0; k < kKvGroups; ++k)
+            ldg_pred(sc[k], a.kv_scale + static_cast<int64_t>(max(my_slot, 0)) * kKvGroups + k, my_slot >= 0);
         }
       }
     };
-    auto store = [&](const uint4 (&raw)[kBatchPieces], int batch, uint8_t* kv, const uint32_t* mult) {
+    auto store = [&](const uint4 (&raw)[kPieces], int batch, uint8_t* kv, const uint32_t* mult, const KVMeta* km) {
       if (FP8) {
 #pragma unroll
-        for (int i = 0; i < kBatchPieces; ++i) {
-          const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
-          const int row = p / kRowPieces, c16 = p - row * kRowPieces;
+        for (int i = 0; i < kPieces; ++i) {
+          const int p = lt + kLoadThreads * (batch * kPieces + i);
+          const int row = PACKED ? packed_row(p) : p / kRowPieces;
+          const int c16 = PACKED ? (p < kPackedCodePieces ? (p & 31) : 32 + (p & 7)) : p - row * kRowPieces;
+          if (PACKED && p >= kPackedCodePieces) {
+            // eight bf16 rope values -> fp16 times 2^-E_j (the row's exponent), in fp32
+            const float inv = exp2i(-km->E[row]);
+            const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+              const __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
+              o[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            *reinterpret_cast<uint4*>(kv + 8 * kKVChunk + swz(row, c16 - 32)) = make_uint4(o[0], o[1], o[2], o[3]);
+            continue;
+          }
           const uint32_t mwi = mult[row * kKvGroups + (c16 >> 3)];
           const __half2 m2 = *reinterpret_cast<const __half2*>(&mwi);
           uint4 o0, o1;
@@ -586,15 +632,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < kBatchPieces; ++i) {
-          const int p = lt + kLoadThreads * (batch * kBatchPieces + i);
+        for (int i = 0; i < kPieces; ++i) {
+          const int p = lt + kLoadThreads * (batch * kPieces + i);
           const int row = p / kRowPieces, c16 = p - row * kRowPieces;
           *reinterpret_cast<uint4*>(kv + (c16 >> 3) * kKVChunk + swz(row, c16 & 7)) = raw[i];
         }
       }
     };
     // one tile: wait for its buffer, publish the row tables, convert, hand over, prefetch T+2
-    auto step = [&](uint4 (&raw)[kBatchPieces], float (&sc)[kKvGroups], int& my_slot, int T) -> bool {
+    auto step = [&](uint4 (&raw)[kPieces], float (&sc)[kKvGroups], int& my_slot, int T) -> bool {
       const int b = T & 1;
       // the buffer was last read by PV(T-2)
       const bool ok = T < 2 || wait_warp(&pv_done[b], ((T >> 1) & 1) ^ 1, abort_flag, a.wait_limit);
@@ -629,10 +675,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
       // also orders this tile's table writes after every loader's reads of tile T-2's
       if (!bar_and(2, kLoadThreads, ok)) return false;
       uint8_t* kv = sKV + b * kKVBytes;
-      store(raw, 0, kv, mult);
+      store(raw, 0, kv, mult, km);
       if (kBatches > 1) {
         fetch(raw, T, 1);
-        store(raw, 1, kv, mult);
+        store(raw, 1, kv, mult, km);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -735,15 +781,17 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
     a.lse[static_cast<int64_t>(q) * kHeads + h] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
-template <bool FP8>
+template <int KVF>
 static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStream_t stream) {
-  cudaError_t e = set_smem_once<mla_decode_kernel<FP8>>(kMlaSmem);
+  cudaError_t e = set_smem_once<mla_decode_kernel<KVF>>(kMlaSmem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(mla_decode_kernel<FP8>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
+  return launch_pdl(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
 }
 
-cudaError_t launch_mla(bool fp8, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
-  cudaError_t e = fp8 ? launch_mla_t<true>(tmap_q, a, stream) : launch_mla_t<false>(tmap_q, a, stream);
+cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
+  cudaError_t e = kvf == kKvFp8Packed ? launch_mla_t<kKvFp8Packed>(tmap_q, a, stream)
+                  : kvf == kKvFp8     ? launch_mla_t<kKvFp8>(tmap_q, a, stream)
+                                      : launch_mla_t<kKvBf16>(tmap_q, a, stream);
   ++*launches;
   if (e != cudaSuccess || a.nsplit == 1) return e;
   ++*launches;

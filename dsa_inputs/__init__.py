@@ -49,7 +49,8 @@ class CaseSpec:
     seq_lens: tuple                  # per-sequence cache lengths
     top_k: int
     idx_dtype: str = "fp8"           # "bf16" | "fp8": indexer q and key cache
-    kv_dtype: str = "fp8"            # "bf16" | "fp8": MLA latent cache
+    kv_dtype: str = "fp8"            # "bf16" | "fp8" | "fp8r": MLA latent cache ("fp8r": packed
+                                     # 656-byte rows, see KV_ROW_FP8R)
     out_dtype: str = "bf16"          # "fp32" | "bf16"
     n_q: int = 1                     # queries per sequence (1 = decode)
     q_pos: Optional[tuple] = None    # causal positions of the n_q queries of a sequence
@@ -89,6 +90,8 @@ CONFIGS = {
     # not one of the five graded configs: the serving workload's rows with three queries
     # each at their last three positions, as a speculative (multi-token) decode verifies them
     "mtp": CaseSpec("mtp", _cfg2_lens(2), top_k=2048, n_q=3, q_tail=True, n_planted=0, seed=5),
+    # not graded either: the serving workload with packed 656-byte latent rows
+    "cfg2r": CaseSpec("cfg2r", _cfg2_lens(2), top_k=2048, kv_dtype="fp8r", n_planted=32, seed=2),
 }
 
 WORKLOAD_NAMES = {
@@ -98,6 +101,7 @@ WORKLOAD_NAMES = {
     "cfg3": "long-context fp8 decode B=1 L=1048576 top_k=2048",
     "cfg4": "chunked-prefill fp8 n_q=2048 at 63488..65535 of L=65536 top_k=2048",
     "mtp": "speculative decode fp8 B=64 L~U[2048,65536] n_q=3 at each row's last 3 positions top_k=2048",
+    "cfg2r": "serving-shaped fp8 decode, packed 656-byte latent rows, B=64 L~U[2048,65536] top_k=2048",
 }
 
 
@@ -220,6 +224,12 @@ def generate(s: CaseSpec) -> dict:
     if s.kv_dtype == "bf16":
         kv_cache = np.full((P * PAGE, DK), to_bf16_bits(np.float32([_POISON_SCALE]))[0], dtype=np.uint16)
         kv_scale = None
+    elif s.kv_dtype == "fp8r":
+        kv_cache = np.empty((P * PAGE, KV_ROW_FP8R), dtype=np.uint8)
+        pack_rows_fp8r(kv_cache, np.full((1, DV), _FP8_POISON, dtype=np.uint8),
+                       np.full((1, 4), _POISON_SCALE, dtype=np.float32),
+                       np.full((1, DK - DV), to_bf16_bits(np.float32([_POISON_SCALE]))[0], dtype=np.uint16))
+        kv_scale = None
     else:
         kv_cache = np.full((P * PAGE, DK), _FP8_POISON, dtype=np.uint8)
         kv_scale = np.full((P * PAGE, KV_GROUPS), _POISON_SCALE, dtype=np.float32)
@@ -264,6 +274,8 @@ def generate(s: CaseSpec) -> dict:
         vf = _rng(s.seed, 5, b, ci).standard_normal((n, DK), dtype=np.float32) * np.float32(s.kv_std)
         if s.kv_dtype == "bf16":
             kv_cache[phys] = to_bf16_bits(vf)
+        elif s.kv_dtype == "fp8r":
+            store_rows_fp8r(kv_cache, phys, vf)
         else:
             groups = [vf[:, g * 128:(g + 1) * 128] for g in range(4)] + [vf[:, 512:576]]
             codes = np.empty((n, DK), dtype=np.uint8)
@@ -330,6 +342,8 @@ def rising_selection(case: dict, tiles: int, climb: float, seed: int = 0, noise_
         rows = rows.astype(np.float32)
         if case["kv_dtype"] == "bf16":
             c["kv_cache"][slots] = to_bf16_bits(rows)
+        elif case["kv_dtype"] == "fp8r":
+            store_rows_fp8r(c["kv_cache"], slots, rows)
         else:
             for g in range(KV_GROUPS):
                 lo, hi = g * 128, min(DK, g * 128 + 128)
@@ -337,6 +351,35 @@ def rising_selection(case: dict, tiles: int, climb: float, seed: int = 0, noise_
                 c["kv_cache"][slots, lo:hi] = codes
                 c["kv_scale"][slots, g] = sc
     return c, phys
+
+
+# Packed fp8 latent rows ("fp8r"), 656 bytes per token: bytes [0, 512) the E4M3 codes of the
+# 512 latent columns, [512, 528) four fp32 scales (one per 128-column group, little-endian),
+# [528, 656) the 64 rope columns as bf16. Storage only: the codes and scales come from
+# quantize_rows_e4m3, the rope bits from to_bf16_bits.
+KV_ROW_FP8R = DV + 4 * 4 + 2 * (DK - DV)
+
+
+def pack_rows_fp8r(dst: np.ndarray, codes: np.ndarray, scales: np.ndarray, rope_bits: np.ndarray, rows=None):
+    """Write packed rows: codes uint8 [n, 512], scales f32 [n, 4], rope bf16 bits [n, 64]
+    into dst[rows] (all rows of dst when rows is None; n = 1 broadcasts)."""
+    sel = slice(None) if rows is None else rows
+    dst[sel, :DV] = codes
+    dst[sel, DV:DV + 16] = np.ascontiguousarray(scales, dtype=np.float32).view(np.uint8).reshape(-1, 16)
+    dst[sel, DV + 16:] = np.ascontiguousarray(rope_bits, dtype=np.uint16).view(np.uint8).reshape(-1, 2 * (DK - DV))
+
+
+def store_rows_fp8r(dst: np.ndarray, rows, vf: np.ndarray):
+    """fp32 rows [n, 576] -> packed fp8r rows at dst[rows]: per-group E4M3 with amax/448
+    scales for the latent columns, bf16 (round to nearest even) for the rope columns."""
+    n = vf.shape[0]
+    codes = np.empty((n, DV), dtype=np.uint8)
+    scs = np.empty((n, 4), dtype=np.float32)
+    for g in range(4):
+        c, sc = quantize_rows_e4m3(vf[:, g * 128:(g + 1) * 128])
+        codes[:, g * 128:(g + 1) * 128] = c
+        scs[:, g] = sc
+    pack_rows_fp8r(dst, codes, scs, to_bf16_bits(vf[:, DV:]), rows)
 
 
 def vis_lengths(case: dict) -> np.ndarray:
@@ -353,7 +396,7 @@ def algorithmic_bytes(case: dict) -> dict:
     MLA row once, every query-side input once and the output once."""
     vis = vis_lengths(case)
     ik = 2 * DI if case["idx_dtype"] == "bf16" else DI + 4
-    kvb = 2 * DK if case["kv_dtype"] == "bf16" else DK + 4 * KV_GROUPS
+    kvb = {"bf16": 2 * DK, "fp8r": KV_ROW_FP8R}.get(case["kv_dtype"], DK + 4 * KV_GROUPS)
     # unique indexer-key bytes: every token of every sequence is read once per call
     lens = case["seq_lens"].astype(np.int64)
     idx_bytes = int(lens.sum()) * ik + int(((lens + PAGE - 1) // PAGE).sum()) * 4
@@ -385,7 +428,7 @@ def to_torch(case: dict, device="cuda") -> dict:
             x = x.view(torch.float8_e4m3fn)
         return x.to(device)
     idk = "bf16" if case["idx_dtype"] == "bf16" else "fp8"
-    kvk = "bf16" if case["kv_dtype"] == "bf16" else "fp8"
+    kvk = {"bf16": "bf16", "fp8": "fp8"}.get(case["kv_dtype"])   # packed fp8r rows stay uint8
     return dict(
         seq_lens=t(case["seq_lens"]), q_pos=t(case["q_pos"]), block_table=t(case["block_table"]),
         q_idx=t(case["q_idx"], idk), q_idx_scale=t(case["q_idx_scale"]), head_w=t(case["head_w"]),

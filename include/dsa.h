@@ -57,7 +57,11 @@ typedef enum {
 typedef enum {
   DSA_BF16 = 0,
   DSA_FP8_E4M3 = 1,
-  DSA_FP32 = 2
+  DSA_FP32 = 2,
+  /* MLA latent caches only: packed 656-byte rows. Bytes [0, 512) the E4M3 codes of the
+   * 512 latent columns; [512, 528) four little-endian fp32 scales, scale g for columns
+   * [128g, 128g+128); [528, 656) the 64 rope columns as bf16. No scale plane. */
+  DSA_FP8_E4M3_ROPE_BF16 = 3
 } dsa_dtype;
 
 /* Which call a workspace is sized for (dsa_workspace_size). */
@@ -142,7 +146,11 @@ dsa_status dsa_pagemap(const dsa_paging* paging, const int32_t* logical, int32_t
  *  q         device [Bq, 64, 576] bf16 (absorbed, post-RoPE query)
  *  kv_cache  device [num_slots, 576] in kv_dtype: DSA_BF16, or DSA_FP8_E4M3 with
  *  kv_scale  device [num_slots, 5] fp32: scale g covers columns [128g, 128g+128) for
- *            g < 4 and the 64 rope columns [512, 576) for g = 4; NULL for bf16
+ *            g < 4 and the 64 rope columns [512, 576) for g = 4; NULL for bf16;
+ *            or kv_cache device [num_slots, 656] bytes in DSA_FP8_E4M3_ROPE_BF16 (the
+ *            packed layout above) with kv_scale NULL. In the packed layout each row's
+ *            values are scaled by 2^-E, E the exponent of its largest group scale, into
+ *            fp16: rope values must stay below 2^16 x 2^E in magnitude
  *  physical  device [Bq, top_k] int32 slots, -1 = unused
  *  out       device [Bq, 64, 512] in out_dtype (DSA_BF16 or DSA_FP32)
  *  lse       device [Bq, 64] fp32 natural-log sum of exp(logits), or NULL

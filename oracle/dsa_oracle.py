@@ -99,11 +99,28 @@ def dequant_index_keys(case: dict, slots: np.ndarray) -> np.ndarray:
     return k
 
 
+def _dequant_packed_rows(rows: np.ndarray) -> np.ndarray:
+    """Packed fp8 latent rows (656 bytes each: the layout variant with bf16 rope columns and
+    four fp32 group scales, "Show HN: colibri", features: 576 values per token = 512 latent +
+    64 rope) -> [n, 576] fp64. Bytes [0, 512): E4M3 codes of the latent columns, column group
+    g = [128g, 128g+128) times the fp32 scale stored little-endian at bytes [512 + 4g,
+    516 + 4g); bytes [528, 656): the 64 rope values as bf16."""
+    rows = np.ascontiguousarray(rows, dtype=np.uint8)
+    n = rows.shape[0]
+    latent = decode_e4m3(rows[:, :DV])                                        # [n, 512]
+    scales = rows[:, DV:DV + 16].copy().view("<f4").astype(np.float64)        # [n, 4]
+    latent = latent * np.repeat(scales, 128, axis=1)
+    rope = decode_bf16(rows[:, DV + 16:].copy().view("<u2").reshape(n, DK - DV))
+    return np.concatenate([latent, rope], axis=1)
+
+
 def dequant_latent_rows(case: dict, slots: np.ndarray) -> np.ndarray:
     """Latent KV rows of the given physical slots, [n, 576] fp64.
 
     fp8 rows: column group g in {0..3} covers columns [128g, 128g+128) and group 4 the
     64 rope columns [512, 576); each group has its own fp32 scale per row."""
+    if case["kv_dtype"] == "fp8r":
+        return _dequant_packed_rows(case["kv_cache"][slots])
     kv = _decode(case["kv_cache"][slots], case["kv_dtype"])
     if case["kv_scale"] is not None:
         sc = case["kv_scale"][slots].astype(np.float64)

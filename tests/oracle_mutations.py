@@ -87,6 +87,20 @@ def _latent_rows_rope_scale_from_group3(case, slots):
     return kv
 
 
+def _packed_rows(scale_shift=0, rope_big_endian=False):
+    def dequant(rows):
+        rows = np.ascontiguousarray(rows, dtype=np.uint8)
+        n = rows.shape[0]
+        latent = od.decode_e4m3(rows[:, :DV])
+        scales = rows[:, DV:DV + 16].copy().view("<f4").astype(np.float64)
+        scales = np.roll(scales, scale_shift, axis=1)
+        latent = latent * np.repeat(scales, 128, axis=1)
+        rope = od.decode_bf16(rows[:, DV + 16:].copy().view(">u2" if rope_big_endian else "<u2").astype(np.uint16)
+                              .reshape(n, DK - DV))
+        return np.concatenate([latent, rope], axis=1)
+    return dequant
+
+
 def _mla(scale_on=True, value_cols=slice(0, DV), key_cols=slice(0, DK), lse_with_max=True):
     def attention(case, physical, queries=None):
         queries = np.arange(physical.shape[0]) if queries is None else np.asarray(queries)
@@ -182,6 +196,7 @@ CONTROLS = {
     "control_topk_copy": lambda: _set("topk_logical", _topk()),
     "control_mla_copy": lambda: _set("mla_sparse_attention", _mla()),
     "control_e4m3_table": lambda: setattr(od, "_E4M3", _e4m3_table()),
+    "control_packed_rows_copy": lambda: _set("_dequant_packed_rows", _packed_rows()),
 }
 
 MUTATIONS = {
@@ -205,6 +220,8 @@ MUTATIONS = {
     "causal_visibility_off_by_one": lambda: _set("visible_lengths", _visible_lengths_causal_off_by_one),
     "pagemap_without_the_page_size": lambda: _set("physical_slots", _physical_slots_without_page_size),
     "mla_softmax_over_heads": lambda: _set("mla_sparse_attention", _mla_softmax_over_heads),
+    "packed_rows_scales_one_group_off": lambda: _set("_dequant_packed_rows", _packed_rows(scale_shift=1)),
+    "packed_rows_rope_big_endian": lambda: _set("_dequant_packed_rows", _packed_rows(rope_big_endian=True)),
 }
 
 

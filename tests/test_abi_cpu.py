@@ -52,6 +52,7 @@ def test_indexer_argument_errors():
     assert call_indexer(pg, qs=None) == dsa.DSA_ERR_INVALID_ARG                      # fp8 needs scales
     assert call_indexer(pg, qd=dsa.DSA_BF16, kd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG  # bf16 takes none
     assert call_indexer(pg, qd=dsa.DSA_FP32, kd=dsa.DSA_FP32) == dsa.DSA_ERR_INVALID_ARG
+    assert call_indexer(pg, qd=dsa.DSA_FP8_E4M3_ROPE_BF16, kd=dsa.DSA_FP8_E4M3_ROPE_BF16) == dsa.DSA_ERR_INVALID_ARG
     assert call_indexer(pg, L=0) == dsa.DSA_ERR_INVALID_ARG
     assert call_indexer(pg, ws_bytes=16) == dsa.DSA_ERR_WORKSPACE
     assert call_indexer(pg, ws=None) == dsa.DSA_ERR_WORKSPACE
@@ -84,6 +85,9 @@ def test_mla_argument_errors():
     assert call(kvd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG
     assert call(outd=dsa.DSA_FP8_E4M3) == dsa.DSA_ERR_INVALID_ARG
     assert call(q=ctypes.c_void_p(0x100008)) == dsa.DSA_ERR_INVALID_ARG   # TMA needs 16-byte alignment
+    # packed 656-byte rows carry their scales: a scale plane is an error
+    assert call(kvd=dsa.DSA_FP8_E4M3_ROPE_BF16) == dsa.DSA_ERR_INVALID_ARG
+    assert call(outd=dsa.DSA_FP8_E4M3_ROPE_BF16) == dsa.DSA_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_are_consistent():

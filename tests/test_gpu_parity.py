@@ -25,6 +25,8 @@ SMALL = {
     # L - n_q + 1 .. L tokens); one row is shorter than top_k and takes the dense path
     "mtp_small": CaseSpec("mtp_small", (300, 1000, 70, 2100), top_k=128, n_q=3, q_tail=True, n_planted=0,
                           seed=38),
+    # packed 656-byte latent rows (E4M3 codes, four fp32 scales, bf16 rope) on ragged rows
+    "packed_fp8": CaseSpec("packed_fp8", (37, 64, 200, 1, 129), top_k=64, kv_dtype="fp8r", seed=40),
     "mtp_bf16": CaseSpec("mtp_bf16", (129, 640), top_k=64, n_q=4, q_tail=True, idx_dtype="bf16", kv_dtype="bf16",
                          out_dtype="fp32", n_planted=0, seed=39),
 }

@@ -38,13 +38,16 @@ CASES = [
     # a gentler climb (a few log2 units per tile) over more tiles
     ("fp8_unsplit_gentle", "fp8", 150, 6, 6.0, 3.2),
     ("fp8_split_gentle", "fp8", 50, 6, 6.0, 3.2),
+    # packed 656-byte rows: the scales grow with the rows, the rope stays bf16
+    ("fp8r_split_steep", "fp8r", 40, 4, 12.0, 8.5),
 ]
 
 
 @functools.lru_cache(maxsize=None)
 def _case(name):
     _, kv, nq, tiles, climb, _ = next(c for c in CASES if c[0] == name)
-    spec = CaseSpec(f"rise_{name}", (tiles * TILE + 37,) * nq, top_k=tiles * TILE, idx_dtype=kv, kv_dtype=kv,
+    spec = CaseSpec(f"rise_{name}", (tiles * TILE + 37,) * nq, top_k=tiles * TILE,
+                    idx_dtype="bf16" if kv == "bf16" else "fp8", kv_dtype=kv,
                     out_dtype="fp32" if kv == "bf16" else "bf16", n_planted=0, seed=61)
     case, phys = rising_selection(generate(spec), tiles, climb, seed=7, noise_std=0.15)
     return case, phys
@@ -86,7 +89,7 @@ def test_mla_matches_oracle_on_rising_logits(name):
     out, lse, err = GpuCase(case).mla(phys)
     assert err == 0
     ref_out, ref_lse = oracle.mla_sparse_attention(case, phys.astype(np.int64))
-    bound = fp8_lse_bound(case, phys) if case["kv_dtype"] == "fp8" else None
+    bound = fp8_lse_bound(case, phys) if case["kv_dtype"] != "bf16" else None
     check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"], lse_bound=bound)
 
 
@@ -101,5 +104,5 @@ def test_mla_matches_oracle_on_falling_logits(name):
     out, lse, err = GpuCase(case).mla(rev)
     assert err == 0
     ref_out, ref_lse = oracle.mla_sparse_attention(case, rev.astype(np.int64))
-    bound = fp8_lse_bound(case, rev) if case["kv_dtype"] == "fp8" else None
+    bound = fp8_lse_bound(case, rev) if case["kv_dtype"] != "bf16" else None
     check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"], lse_bound=bound)

@@ -7,6 +7,8 @@ import json
 import math
 import os
 
+import struct
+
 import numpy as np
 import pytest
 import torch
@@ -46,6 +48,61 @@ def test_bf16_decode_vs_torch():
     bits = bits[exp != 0xFF]                      # leave out inf/nan patterns
     ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
     assert np.array_equal(oracle.decode_bf16(bits), ref)
+
+
+def _packed_rows(codes, scales, rope):
+    """656-byte packed latent rows built byte by byte: codes, the four scales as
+    little-endian fp32 (struct), the rope values encoded to bf16 by PyTorch."""
+    n = codes.shape[0]
+    rows = np.zeros((n, 656), dtype=np.uint8)
+    rows[:, :512] = codes
+    rows[:, 512:528] = np.frombuffer(struct.pack("<4f", *[float(x) for x in scales]), dtype=np.uint8)
+    bits = torch.from_numpy(np.ascontiguousarray(rope, dtype=np.float32)).to(torch.bfloat16).view(torch.int16)
+    rows[:, 528:] = bits.numpy().astype("<i2").view(np.uint8).reshape(n, 128)
+    return rows
+
+
+def test_packed_rows_decode_by_their_byte_layout():
+    """The packed fp8 latent row (656 bytes, the layout variant with bf16 rope columns):
+    E4M3 codes of the 512 latent columns, one fp32 scale per 128-column group at bytes
+    512..527, then the 64 rope values in bf16. Codes are decoded by PyTorch, the column
+    ranges written out by hand."""
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, size=(64, 512)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C                       # no NaN codes
+    scales = np.array([0.5, 2.0, 4.0, 8.0], dtype=np.float32)
+    rope = rng.standard_normal((64, 64)).astype(np.float32)
+    case = dict(kv_cache=_packed_rows(codes, scales, rope), kv_scale=None, kv_dtype="fp8r")
+    got = oracle.dequant_latent_rows(case, np.arange(64))
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for g, (lo, hi) in enumerate([(0, 128), (128, 256), (256, 384), (384, 512)]):
+        assert np.array_equal(got[:, lo:hi], vals[:, lo:hi] * float(scales[g])), g
+    want_rope = torch.from_numpy(rope).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got[:, 512:], want_rope)
+
+
+def test_packed_rows_agree_with_the_scale_plane_layout():
+    """Where the rope values are exact in both formats (E4M3 codes times a power of two),
+    a packed row and a row of the five-scale layout hold the same numbers, and attention
+    over them is identical."""
+    rng = np.random.default_rng(6)
+    codes = rng.integers(0, 0x7F, size=(64, DK)).astype(np.uint8)
+    scales = np.array([0.25, 0.5, 1.0, 2.0, 0.125], dtype=np.float32)
+    plane = blank_case((64,), top_k=64, idx_dtype="fp8", kv_dtype="fp8")
+    plane["kv_cache"][:64] = codes
+    plane["kv_scale"][:64] = scales
+    rope = torch.from_numpy(codes[:, 512:]).view(torch.float8_e4m3fn).to(torch.float64).numpy() * 0.125
+    packed = dict(plane, kv_cache=_packed_rows(codes[:, :512], scales[:4], rope), kv_scale=None, kv_dtype="fp8r")
+    slots = np.arange(64)
+    assert np.array_equal(oracle.dequant_latent_rows(packed, slots), oracle.dequant_latent_rows(plane, slots))
+    q = rng.standard_normal((1, H, DK)).astype(np.float32)
+    qb = torch.from_numpy(q).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    plane["q_mla"] = qb
+    packed["q_mla"] = qb
+    phys = slots[None, :].astype(np.int64)
+    o1, l1 = oracle.mla_sparse_attention(plane, phys)
+    o2, l2 = oracle.mla_sparse_attention(packed, phys)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
 def test_scales_apply_to_their_columns():
