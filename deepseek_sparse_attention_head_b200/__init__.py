@@ -63,6 +63,8 @@ _SIGNATURES = {
                                          _vp]),
     "dsa_decode_layer": (_i32, [_PP, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _f32, _vp, _i32,
                                 _vp, _vp, _vp, _vp, _sz, _vp]),
+    "dsa_rope_quantize_append": (_i32, [_PP, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
+                                        _vp]),
     "dsa_workspace_size": (_sz, [_PP, _i64, _i32, _i32]),
     "mla_workspace_size": (_sz, [_i32, _i32]),
     "mla_num_splits": (_i32, [_i32, _i32]),
@@ -226,6 +228,21 @@ def dsa_pagemap(paging: Paging, logical: torch.Tensor, physical: torch.Tensor, w
                           workspace.numel(), _stream(stream))
     _check(st, "dsa_pagemap")
     return physical
+
+
+def dsa_rope_quantize_append(paging: Paging, idx_q: torch.Tensor, idx_k: torch.Tensor, latent: torch.Tensor,
+                             q_mla, q_idx_out: torch.Tensor, q_scale_out: torch.Tensor, k_cache: torch.Tensor,
+                             k_scale: torch.Tensor, kv_cache: torch.Tensor, kv_scale, rope_base: float = 10000.0,
+                             status=None, stream=None):
+    """The step before the path for every query's new token (see include/dsa.h): RoPE on
+    the rope columns, E4M3 quantisation, and the key and latent rows written at the
+    token's cache slot. Returns (q_idx_out, q_scale_out)."""
+    st = _lib.dsa_rope_quantize_append(paging.ref(), _ptr(idx_q), _ptr(idx_k), _ptr(latent), _ptr(q_mla),
+                                       float(rope_base), _ptr(q_idx_out), _ptr(q_scale_out), _ptr(k_cache),
+                                       _ptr(k_scale), _ptr(kv_cache), _kv_code(kv_cache), _ptr(kv_scale),
+                                       _ptr(status), _stream(stream))
+    _check(st, "dsa_rope_quantize_append")
+    return q_idx_out, q_scale_out
 
 
 def mla_sparse_decode(q: torch.Tensor, kv_cache: torch.Tensor, kv_scale, physical: torch.Tensor,

@@ -90,7 +90,7 @@ int mla_splits_for(int Bq, int top_k, int* keys_per_split, int max_ctas = 0) {
   const int ntiles = (top_k + tile - 1) / tile;
   const int64_t bq = Bq > 0 ? Bq : 1;
   const int64_t cap = max_ctas > 0 ? std::max<int64_t>(max_ctas, bq) : std::max<int64_t>(4LL * sms, bq);
-  int best_s = 1, best_tiles = ntiles;
+  int best_tiles = ntiles;
   int64_t best_cost = -1;
   for (int s = 1; s <= ntiles; ++s) {
     const int tps = (ntiles + s - 1) / s;           // tiles per split
@@ -101,7 +101,6 @@ int mla_splits_for(int Bq, int top_k, int* keys_per_split, int max_ctas = 0) {
     const int64_t cost = waves * (tps + kFixedTiles + (se > 1 ? 1 : 0));
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best_s = se;
       best_tiles = tps;
     }
   }
@@ -542,4 +541,56 @@ extern "C" dsa_status mla_sparse_decode_noalloc(int32_t Bq, const void* q, const
               scratch, lay, nsplit, kps, st);
   if (s != DSA_OK || status == nullptr) return s;
   return cuda_status(cudaMemcpyAsync(status, scratch, 8, cudaMemcpyDeviceToDevice, st));
+}
+
+// ====================================================================== the step before the path
+
+extern "C" dsa_status dsa_rope_quantize_append(const dsa_paging* paging, const void* idx_q, const void* idx_k,
+                                               const void* latent, void* q_mla, float rope_base, void* q_idx_out,
+                                               float* q_scale_out, void* k_cache, float* k_scale, void* kv_cache,
+                                               dsa_dtype kv_dtype, float* kv_scale, unsigned int* status,
+                                               void* stream) {
+  g_launches = 0;
+  dsa_status s = check_paging(paging);
+  if (s != DSA_OK) return s;
+  if (idx_q == nullptr || idx_k == nullptr || latent == nullptr || q_idx_out == nullptr || q_scale_out == nullptr ||
+      k_cache == nullptr || k_scale == nullptr || kv_cache == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  if (!(rope_base > 1.0f) || !std::isfinite(rope_base)) return DSA_ERR_INVALID_ARG;
+  int kvf = kKvBf16;
+  if (kv_dtype == DSA_FP8_E4M3) {
+    if (kv_scale == nullptr || !aligned(kv_scale, 4)) return DSA_ERR_INVALID_ARG;
+    kvf = kKvFp8;
+  } else if (kv_dtype == DSA_FP8_E4M3_ROPE_BF16 || kv_dtype == DSA_BF16) {
+    if (kv_scale != nullptr) return DSA_ERR_INVALID_ARG;
+    kvf = kv_dtype == DSA_BF16 ? kKvBf16 : kKvFp8Packed;
+  } else {
+    return DSA_ERR_INVALID_ARG;
+  }
+  if (!aligned(idx_q, 16) || !aligned(idx_k, 16) || !aligned(latent, 16) || !aligned(q_idx_out, 16) ||
+      !aligned(q_scale_out, 4) || !aligned(k_cache, 16) || !aligned(k_scale, 4) || !aligned(kv_cache, 16) ||
+      (q_mla != nullptr && !aligned(q_mla, 16)) || (status != nullptr && !aligned(status, 8)))
+    return DSA_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.n_q = paging->n_q;
+  a.seq_lens = paging->seq_lens;
+  a.q_pos = paging->q_pos;
+  a.block_table = paging->block_table;
+  a.max_pages = paging->max_pages_per_seq;
+  a.num_pages = paging->num_pages;
+  a.idx_q = static_cast<const uint16_t*>(idx_q);
+  a.idx_k = static_cast<const uint16_t*>(idx_k);
+  a.latent = static_cast<const uint16_t*>(latent);
+  a.q_mla = static_cast<uint16_t*>(q_mla);
+  a.rope_base = rope_base;
+  a.q_out = static_cast<uint8_t*>(q_idx_out);
+  a.q_scale_out = q_scale_out;
+  a.k_cache = static_cast<uint8_t*>(k_cache);
+  a.k_scale = k_scale;
+  a.kv_cache = kv_cache;
+  a.kvf = kvf;
+  a.kv_scale = kv_scale;
+  a.err = status;
+  const int Bq = paging->B * paging->n_q;
+  return cuda_status(launch_rope_quantize_append(a, Bq, static_cast<cudaStream_t>(stream), &g_launches));
 }

@@ -47,6 +47,31 @@ struct TopkArgs {
   int32_t* g_idx;
 };
 
+// The step before the path (append.cu): each query's new token at position q_pos[q] (or
+// seq_lens[b] - 1). Inputs are bf16 bit patterns; kvf is one of kKvBf16 / kKvFp8 /
+// kKvFp8Packed (declared below).
+struct AppendArgs {
+  int n_q;
+  const int32_t* seq_lens;
+  const int32_t* q_pos;
+  const int32_t* block_table;
+  int max_pages;
+  int num_pages;
+  const uint16_t* idx_q;    // [Bq, 64, 128]
+  const uint16_t* idx_k;    // [Bq, 128]
+  const uint16_t* latent;   // [Bq, 576]
+  uint16_t* q_mla;          // [Bq, 64, 576] (rope columns rotated in place) or null
+  float rope_base;
+  uint8_t* q_out;           // [Bq, 64, 128] e4m3
+  float* q_scale_out;       // [Bq, 64]
+  uint8_t* k_cache;         // [num_pages * 64, 128] e4m3
+  float* k_scale;           // [num_pages * 64]
+  void* kv_cache;
+  int kvf;
+  float* kv_scale;          // [num_pages * 64, 5] (kKvFp8 only)
+  unsigned int* err;
+};
+
 // Per-(query, split, head) partial statistics: m, l, then one normaliser per value group.
 constexpr int kPartStats = 6;
 
@@ -125,6 +150,7 @@ cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* blo
 constexpr int kKvBf16 = 0, kKvFp8 = 1, kKvFp8Packed = 2;
 constexpr int kPackedRowBytes = kDimV + 4 * 4 + 2 * (kDimK - kDimV);
 cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches);
+cudaError_t launch_rope_quantize_append(const AppendArgs& a, int Bq, cudaStream_t stream, int* launches);
 int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
 }  // namespace dsa

@@ -435,3 +435,22 @@ def to_torch(case: dict, device="cuda") -> dict:
         k_cache=t(case["k_cache"], idk), k_scale=t(case["k_scale"]),
         q_mla=t(case["q_mla"], "bf16"), kv_cache=t(case["kv_cache"], kvk), kv_scale=t(case["kv_scale"]),
     )
+
+
+def new_token_inputs(case: dict, seed: int = 0, with_q_mla: bool = True) -> dict:
+    """Projected, pre-RoPE inputs of every query's new token, as bf16 bit patterns:
+    idx_q [Bq, 64, 128] ~ N(0, 1/128) (like the indexer queries), idx_k [Bq, 128] ~ N(0, 1/128),
+    latent [Bq, 576] ~ kv_std * N(0, 1) (like the cached rows) and q_mla [Bq, 64, 576] ~ N(0, 1).
+    Input recipe only (seeded draws), no arithmetic of the method."""
+    s = case["spec"] if "spec" in case else None
+    kv_std = s.kv_std if s is not None else 0.5
+    Bq = case["Bq"]
+    r = _rng(seed, 41)
+    out = dict(
+        idx_q=to_bf16_bits(r.standard_normal((Bq, H, DI), dtype=np.float32) / np.float32(math.sqrt(DI))),
+        idx_k=to_bf16_bits(r.standard_normal((Bq, DI), dtype=np.float32) / np.float32(math.sqrt(DI))),
+        latent=to_bf16_bits(r.standard_normal((Bq, DK), dtype=np.float32) * np.float32(kv_std)),
+    )
+    if with_q_mla:
+        out["q_mla"] = to_bf16_bits(r.standard_normal((Bq, H, DK), dtype=np.float32))
+    return out

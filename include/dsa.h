@@ -231,6 +231,36 @@ const char* dsa_status_string(dsa_status status);
 int32_t dsa_last_launch_count(void);
 
 /*
+ * The step before the decode path, for each query's new token (the position q_pos[q], or
+ * seq_lens[b] - 1 when q_pos is NULL; the token's row must already be counted in
+ * seq_lens): partial interleaved RoPE ("Show HN: colibri", features: MLA attention with
+ * partial interleaved RoPE) on the 64 rope columns of the projected indexer query (the
+ * first 64 of each head's 128), the indexer key (the first 64 of 128) and the latent row
+ * (columns 512..575), pair i of them turned by pos * rope_base^(-2i/64); E4M3
+ * quantisation with amax/448 fp32 scales (1 for an all-zero vector), one per (query,
+ * head), one per key, one per 128-column latent group (plus one for the rope columns in
+ * DSA_FP8_E4M3); and the key and latent rows written at the token's slot
+ * block_table[b, pos / 64] * 64 + pos % 64 of the paged caches.
+ *  idx_q      device [Bq, 64, 128] bf16, idx_k [Bq, 128] bf16, latent [Bq, 576] bf16
+ *             (projected, before RoPE; 16-byte aligned)
+ *  q_mla      device [Bq, 64, 576] bf16 absorbed MLA queries, columns 512..575 rotated
+ *             in place; or NULL
+ *  q_idx_out  device [Bq, 64, 128] e4m3 and q_scale_out [Bq, 64] fp32: the indexer's
+ *             query inputs (q_idx, q_scale of dsa_indexer_scores)
+ *  k_cache    device [num_pages, 64, 128] e4m3 with k_scale [num_pages, 64] fp32
+ *  kv_cache   device latent cache in kv_dtype: DSA_FP8_E4M3 with kv_scale [slots, 5],
+ *             DSA_FP8_E4M3_ROPE_BF16 (656-byte rows) or DSA_BF16, kv_scale NULL
+ *  status     optional device [2] uint32 (8-byte aligned, zero before the call): receives
+ *             DSA_ERR_DEVICE_BOUNDS for a position or page outside the table; that
+ *             token's cache rows are then not written
+ * Two queries must not name the same slot. Out-of-place, no workspace, one launch.
+ */
+dsa_status dsa_rope_quantize_append(const dsa_paging* paging, const void* idx_q, const void* idx_k,
+                                    const void* latent, void* q_mla, float rope_base, void* q_idx_out,
+                                    float* q_scale_out, void* k_cache, float* k_scale, void* kv_cache,
+                                    dsa_dtype kv_dtype, float* kv_scale, unsigned int* status, void* stream);
+
+/*
  * Test hook for the bounded waits of the fp8-cache MLA decode kernel (the kernel
  * mla_sparse_decode, mla_sparse_decode_noalloc and dsa_decode_layer run for an fp8 latent
  * cache). It applies to the later calls made on this host thread.

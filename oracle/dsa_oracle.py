@@ -29,6 +29,14 @@ format, page size or tie rule; these are the plainest readings the rest supports
   * ties in top-k go to the lower logical index; output is in descending-score order;
   * with vis(q) <= top_k every visible token is selected (the dense path);
   * an empty selection gives a zero output and lse = -inf.
+
+The step before the path (rope_quantize_append, the next step after the hot path): the new
+tokens' projected indexer queries and keys and latent rows get partial interleaved RoPE
+("Show HN: colibri", features: MLA with partial interleaved RoPE) on their 64 rope columns
+(the first 64 of the 128 indexer dims, the last 64 of the 576 latent columns), are
+quantised to E4M3 with amax/448 fp32 scales (one per query head, one per key, one per
+latent column group), and the keys and latent rows are written into the paged caches at
+the token's slot.
 """
 from __future__ import annotations
 
@@ -72,6 +80,38 @@ def decode_bf16(bits: np.ndarray) -> np.ndarray:
     """bfloat16 bit pattern -> exact fp64 value (bf16 is the top half of an IEEE fp32)."""
     b = np.asarray(bits).astype(np.uint32) << np.uint32(16)
     return b.view(np.float32).astype(np.float64)
+
+
+def encode_e4m3(x: np.ndarray) -> np.ndarray:
+    """E4M3 codes of finite values (OCP 8-bit floating point): the nearest representable
+    magnitude, ties to the even code (mantissa LSB 0), saturating at 448; the sign bit
+    follows the sign of x (so -0 and small negatives give 0x80)."""
+    x = np.asarray(x, dtype=np.float64)
+    pos_vals = _E4M3[:0x7F]                       # codes 0x00 .. 0x7E, increasing, 0 .. 448
+    m = np.minimum(np.abs(x), pos_vals[-1])
+    hi = np.clip(np.searchsorted(pos_vals, m, side="left"), 0, 0x7E)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = m - pos_vals[lo], pos_vals[hi] - m
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(take_hi, hi, lo).astype(np.uint8)
+    return np.where(np.signbit(x), code | np.uint8(0x80), code).astype(np.uint8)
+
+
+def quantize_e4m3(x: np.ndarray):
+    """amax / 448 scaling along the last axis, stored as fp32 (1 for an all-zero row), and
+    the E4M3 codes of x / scale (fp64 division by the stored scale) -> (codes, scales)."""
+    x = np.asarray(x, dtype=np.float64)
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / 448.0, 1.0).astype(np.float32)
+    return encode_e4m3(x / scale.astype(np.float64)[..., None]), scale
+
+
+def encode_bf16(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of finite fp64 values: round to nearest even on the fp32 value's
+    low 16 bits (the fp64 -> fp32 step rounds to nearest too)."""
+    u = np.asarray(x, dtype=np.float64).astype(np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    return ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint16)
 
 
 def _decode(codes: np.ndarray, dtype: str) -> np.ndarray:
@@ -294,3 +334,85 @@ def decode_layer(case: dict, queries=None):
         phys[i] = physical_slots(case["block_table"][q // case["n_q"]], logical[i])
     out, lse = mla_sparse_attention(case, phys, queries)
     return dict(scores=scores, logical=logical, physical=phys, out=out, lse=lse)
+
+
+# ----------------------------------------------------------------------------------
+# the step before the path: partial interleaved RoPE, fp8 quantise-and-append
+
+ROPE_DIMS = 64
+
+
+def rope_interleaved(x: np.ndarray, pos, base: float = 10000.0) -> np.ndarray:
+    """Rotates consecutive pairs (x[2i], x[2i+1]) of the last axis (n = 64 rope columns) by
+    pos * base^(-2i / n): x'[2i] = x[2i] cos - x[2i+1] sin, x'[2i+1] = x[2i] sin + x[2i+1] cos.
+    `pos` broadcasts against x's leading axes."""
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    theta = base ** (-2.0 * np.arange(n // 2) / n)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    c, s = np.cos(ang), np.sin(ang)
+    out = np.empty_like(x)
+    xe, xo = x[..., 0::2], x[..., 1::2]
+    out[..., 0::2] = xe * c - xo * s
+    out[..., 1::2] = xe * s + xo * c
+    return out
+
+
+def new_token_positions(case: dict) -> np.ndarray:
+    """Position of each query's new token: q_pos when given, else the row's last token."""
+    if case.get("q_pos") is not None:
+        return case["q_pos"].astype(np.int64)
+    return np.repeat(case["seq_lens"].astype(np.int64) - 1, case["n_q"])
+
+
+def physical_slots_rows(case: dict, rows: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """Slot of token pos[i] of sequence rows[i]: table[row, pos // 64] * 64 + pos % 64."""
+    bt = case["block_table"]
+    return bt[rows, pos // PAGE].astype(np.int64) * PAGE + pos % PAGE
+
+
+def rope_quantize_append(case: dict, new: dict, base: float = 10000.0) -> dict:
+    """The step before the path for every query's new token. `new` holds the projected,
+    pre-RoPE bf16 bit tensors idx_q [Bq, 64, 128], idx_k [Bq, 128], latent [Bq, 576] and
+    optionally q_mla [Bq, 64, 576]. Returns
+      q_codes [Bq, 64, 128] e4m3, q_scale [Bq, 64] f32   (the indexer queries);
+      slots [Bq]                                          (where the new token's rows go);
+      k_codes [Bq, 128], k_scale [Bq]                     (the index-cache rows);
+      the latent rows in the case's format: latent_codes [Bq, 576] + latent_scales [Bq, 5]
+        ("fp8"), latent_packed [Bq, 656] bytes ("fp8r") or latent_bf16 [Bq, 576] ("bf16");
+      q_mla [Bq, 64, 576] bf16 bits with its rope columns rotated (when given)."""
+    pos = new_token_positions(case)
+    b = np.arange(case["Bq"]) // case["n_q"]
+    R = ROPE_DIMS
+    q = decode_bf16(new["idx_q"])
+    q[..., :R] = rope_interleaved(q[..., :R], pos[:, None], base)
+    q_codes, q_scale = quantize_e4m3(q)
+    k = decode_bf16(new["idx_k"])
+    k[..., :R] = rope_interleaved(k[..., :R], pos, base)
+    k_codes, k_scale = quantize_e4m3(k)
+    lat = decode_bf16(new["latent"])
+    lat[..., DV:] = rope_interleaved(lat[..., DV:], pos, base)
+    out = dict(q_codes=q_codes, q_scale=q_scale, slots=physical_slots_rows(case, b, pos),
+               k_codes=k_codes, k_scale=k_scale)
+    kvd = case["kv_dtype"]
+    if kvd == "bf16":
+        out["latent_bf16"] = encode_bf16(lat)
+    else:
+        groups = [(128 * g, 128 * g + 128) for g in range(4)] + [(DV, DK)]
+        codes = np.zeros(lat.shape, dtype=np.uint8)
+        scales = np.zeros((lat.shape[0], 5), dtype=np.float32)
+        for g, (lo, hi) in enumerate(groups[:5 if kvd == "fp8" else 4]):
+            codes[:, lo:hi], scales[:, g] = quantize_e4m3(lat[:, lo:hi])
+        if kvd == "fp8":
+            out["latent_codes"], out["latent_scales"] = codes, scales
+        else:
+            row = np.zeros((lat.shape[0], DV + 16 + 2 * (DK - DV)), dtype=np.uint8)
+            row[:, :DV] = codes[:, :DV]
+            row[:, DV:DV + 16] = scales[:, :4].astype("<f4").view(np.uint8).reshape(-1, 16)
+            row[:, DV + 16:] = encode_bf16(lat[:, DV:]).astype("<u2").view(np.uint8).reshape(-1, 2 * (DK - DV))
+            out["latent_packed"] = row
+    if new.get("q_mla") is not None:
+        qm = decode_bf16(new["q_mla"])
+        qm[..., DV:] = rope_interleaved(qm[..., DV:], pos[:, None], base)
+        out["q_mla"] = encode_bf16(qm)
+    return out

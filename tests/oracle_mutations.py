@@ -227,3 +227,28 @@ MUTATIONS = {
 
 def apply(name):
     (MUTATIONS.get(name) or CONTROLS[name])()
+
+
+def _rope_half_split(x, pos, base=10000.0):
+    x = np.asarray(x, dtype=np.float64)
+    n = x.shape[-1]
+    theta = base ** (-2.0 * np.arange(n // 2) / n)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * theta
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., :n // 2], x[..., n // 2:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def _rope_reversed(x, pos, base=10000.0):
+    return _ORIG_ROPE(x, -np.asarray(pos, dtype=np.float64), base)
+
+
+def _slots_one_page_off(case, rows, pos):
+    bt = case["block_table"]
+    return bt[rows, np.minimum(pos // PAGE + 1, bt.shape[1] - 1)].astype(np.int64) * PAGE + pos % PAGE
+
+
+_ORIG_ROPE = od.rope_interleaved
+MUTATIONS["rope_rotates_halves_not_pairs"] = lambda: _set("rope_interleaved", _rope_half_split)
+MUTATIONS["rope_turns_the_other_way"] = lambda: _set("rope_interleaved", _rope_reversed)
+MUTATIONS["append_slot_one_page_off"] = lambda: _set("physical_slots_rows", _slots_one_page_off)

@@ -131,3 +131,23 @@ def test_wait_hook_argument_errors():
     assert _lib.dsa_test_set_wait_hooks(0, 2) == dsa.DSA_ERR_INVALID_ARG
     assert _lib.dsa_test_set_wait_hooks(1000, 1) == dsa.DSA_OK
     assert _lib.dsa_test_set_wait_hooks(0, 0) == dsa.DSA_OK
+
+
+def test_append_argument_errors():
+    pg = paging(B=2, n_q=1, max_pages=4)
+
+    def call(idx_q=FAKE, kvd=dsa.DSA_FP8_E4M3, kvs=FAKE, base=10000.0, status=None, q_mla=None):
+        return _lib.dsa_rope_quantize_append(ctypes.byref(pg), idx_q, FAKE, FAKE, q_mla, base, FAKE, FAKE, FAKE,
+                                             FAKE, FAKE, kvd, kvs, status, None)
+    assert call(idx_q=None) == dsa.DSA_ERR_INVALID_ARG
+    assert call(kvs=None) == dsa.DSA_ERR_INVALID_ARG                               # fp8 needs its scale plane
+    assert call(kvd=dsa.DSA_FP8_E4M3_ROPE_BF16) == dsa.DSA_ERR_INVALID_ARG          # packed rows take none
+    assert call(kvd=dsa.DSA_BF16) == dsa.DSA_ERR_INVALID_ARG
+    assert call(kvd=dsa.DSA_FP32) == dsa.DSA_ERR_INVALID_ARG
+    assert call(base=1.0) == dsa.DSA_ERR_INVALID_ARG
+    assert call(base=float("inf")) == dsa.DSA_ERR_INVALID_ARG
+    assert call(idx_q=ctypes.c_void_p(0x100008)) == dsa.DSA_ERR_INVALID_ARG         # 16-byte alignment
+    assert call(q_mla=ctypes.c_void_p(0x100008)) == dsa.DSA_ERR_INVALID_ARG
+    assert call(status=ctypes.c_void_p(0x100004)) == dsa.DSA_ERR_INVALID_ARG
+    assert _lib.dsa_rope_quantize_append(None, FAKE, FAKE, FAKE, None, 10000.0, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                         dsa.DSA_FP8_E4M3, FAKE, None, None) == dsa.DSA_ERR_INVALID_ARG

@@ -425,3 +425,83 @@ def test_poison_never_reaches_outputs():
     case = generate(CaseSpec("t", (70,), top_k=128, seed=29))
     r = oracle.decode_layer(case)
     assert np.all(np.abs(r["out"]) < 10)
+
+
+# ---------------------------------------------------------------- the step before the path
+
+def test_e4m3_encoder_round_trips_ties_to_even_and_saturates():
+    """Every finite code's value encodes back to that code; the midpoint of two adjacent
+    magnitudes goes to the even code; magnitudes past 448 saturate; random values agree
+    with PyTorch's float8_e4m3fn conversion."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = oracle.decode_e4m3(codes)
+    got = oracle.encode_e4m3(vals)
+    zero = vals == 0
+    assert np.array_equal(got[~zero], codes[~zero])
+    pos = oracle.decode_e4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = (pos[:-1] + pos[1:]) / 2
+    want = np.where(np.arange(1, 0x7F) % 2 == 0, np.arange(1, 0x7F), np.arange(0, 0x7E)).astype(np.uint8)
+    assert np.array_equal(oracle.encode_e4m3(mids), want)
+    assert oracle.encode_e4m3(np.array([1e6, -500.0])).tolist() == [0x7E, 0xFE]
+    x = np.random.default_rng(11).standard_normal(50000) * 60
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.encode_e4m3(x.astype(np.float32).astype(np.float64)), ref)
+
+
+def test_bf16_encoder_matches_torch_and_keeps_bf16_values():
+    x = np.random.default_rng(12).standard_normal(50000).astype(np.float32) * 7
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.encode_bf16(x.astype(np.float64)), ref)
+    exact = oracle.decode_bf16(ref)
+    assert np.array_equal(oracle.encode_bf16(exact), ref)
+
+
+def test_rope_interleaved_by_hand_and_by_its_invariants():
+    """pos 0 is the identity; each pair keeps its norm; rotations compose (p1 then p2 is
+    p1 + p2); a unit vector in pair 0 turns by pos radians (theta_0 = 1) and one in pair 16
+    by pos / 100 (theta_16 = 10000^(-1/2))."""
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((5, 64))
+    assert np.array_equal(oracle.rope_interleaved(x, np.zeros(5)), x)
+    y = oracle.rope_interleaved(x, np.arange(5) * 1000.0 + 3)
+    assert np.allclose(np.hypot(y[:, 0::2], y[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]), atol=1e-12)
+    two = oracle.rope_interleaved(oracle.rope_interleaved(x, 17.0), 40.0)
+    assert np.allclose(two, oracle.rope_interleaved(x, 57.0), atol=1e-12)
+    e = np.zeros((2, 64))
+    e[0, 0] = 1.0
+    e[1, 32] = 1.0
+    r = oracle.rope_interleaved(e, np.array([2.5, 300.0]))
+    assert np.allclose(r[0, :2], [math.cos(2.5), math.sin(2.5)], atol=1e-15)
+    assert np.allclose(r[1, 32:34], [math.cos(3.0), math.sin(3.0)], atol=1e-12)
+    assert np.count_nonzero(r[0, 2:]) == 0 and np.count_nonzero(r[1, :32]) == 0
+
+
+def test_quantize_maps_amax_to_448_and_zero_rows_to_scale_one():
+    x = np.array([[0.5, -2.0, 1.0], [0.0, 0.0, 0.0]])
+    codes, scale = oracle.quantize_e4m3(x)
+    assert scale.dtype == np.float32 and scale.tolist() == [np.float32(2.0 / 448.0), 1.0]
+    assert codes[0, 1] == 0xFE and codes[1].tolist() == [0, 0, 0]
+
+
+def test_rope_quantize_append_slots_and_untouched_columns():
+    """The new token of each row goes to table[row, pos // 64] * 64 + pos % 64 (a permuted
+    table, written out by hand); the non-rope columns are plain quantisations of the
+    inputs; the MLA query keeps its 512 latent columns bit for bit."""
+    table = np.array([[3, 0, -1], [1, 2, 4]], dtype=np.int32)
+    case = blank_case((70, 150), idx_dtype="fp8", kv_dtype="fp8", max_pages=3, table=table)
+    assert oracle.new_token_positions(case).tolist() == [69, 149]
+    rng = np.random.default_rng(14)
+    new = dict(idx_q=bf16(rng.standard_normal((2, H, DI))), idx_k=bf16(rng.standard_normal((2, DI))),
+               latent=bf16(rng.standard_normal((2, DK))), q_mla=bf16(rng.standard_normal((2, H, DK))))
+    r = oracle.rope_quantize_append(case, new)
+    assert r["slots"].tolist() == [0 * 64 + 5, 4 * 64 + 21]
+    k = oracle.decode_bf16(new["idx_k"])
+    # the key's columns 64.. are not rotated: their codes are those of x / (the row's scale)
+    want = oracle.encode_e4m3(k[:, 64:] / r["k_scale"].astype(np.float64)[:, None])
+    assert np.array_equal(r["k_codes"][:, 64:], want)
+    assert np.array_equal(r["q_mla"][..., :DV], new["q_mla"][..., :DV])
+    lat = oracle.decode_bf16(new["latent"])
+    for g in range(4):
+        codes, scale = oracle.quantize_e4m3(lat[:, 128 * g:128 * g + 128])
+        assert np.array_equal(r["latent_codes"][:, 128 * g:128 * g + 128], codes)
+        assert np.array_equal(r["latent_scales"][:, g], scale)
