@@ -582,7 +582,7 @@ extern "C" dsa_status dsa_rope_quantize_append(const dsa_paging* paging, const v
   a.idx_k = static_cast<const uint16_t*>(idx_k);
   a.latent = static_cast<const uint16_t*>(latent);
   a.q_mla = static_cast<uint16_t*>(q_mla);
-  a.rope_base = rope_base;
+  for (int i = 0; i < 32; ++i) a.theta[i] = std::pow(static_cast<double>(rope_base), -2.0 * i / 64.0);
   a.q_out = static_cast<uint8_t*>(q_idx_out);
   a.q_scale_out = q_scale_out;
   a.k_cache = static_cast<uint8_t*>(k_cache);

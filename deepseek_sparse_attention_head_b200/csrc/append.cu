@@ -7,8 +7,9 @@
 // the token's slot. The absorbed MLA query's rope columns are rotated in place as well.
 //
 // One CTA of 256 threads per new token. Pair i of the rope columns turns by
-// pos * base^(-2i/64); the 32 angles are formed and reduced in fp64 (positions reach 1M),
-// then rotated in fp32 like every other step.
+// pos * base^(-2i/64): the frequencies come from the host in fp64, each angle is formed and
+// reduced to [-pi, pi] in fp64 (positions reach 1M), and its cosine and sine are taken in
+// fp32 from there, like every later step of the rotation.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -50,8 +51,35 @@ __global__ void __launch_bounds__(kAppThreads) rope_quantize_append_kernel(const
   pdl_trigger();
   pdl_wait();
 
-  // ---- the token's position and slot (no cache write when either is out of range)
+  // ---- every row this thread reads, issued before the position -> page lookup so that the
+  // loads and that dependent pair of reads overlap
   int pos = a.q_pos != nullptr ? a.q_pos[q] : a.seq_lens[b] - 1;
+  const int h = t >> 2, part = t & 3;
+  uint4 qw[4];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.idx_q + (static_cast<int64_t>(q) * kHeads + h) * kDimIdx +
+                                                      32 * part);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qw[i] = src[i];
+  }
+  const uint32_t kw = t < 64 ? reinterpret_cast<const uint32_t*>(a.idx_k + static_cast<int64_t>(q) * kDimIdx)[t] : 0u;
+  uint32_t lw[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int p = t + kAppThreads * k;
+    lw[k] = p < kDimK / 2 ? reinterpret_cast<const uint32_t*>(a.latent + static_cast<int64_t>(q) * kDimK)[p] : 0u;
+  }
+  uint32_t mw[8];
+  if (a.q_mla != nullptr) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int j = t + kAppThreads * k;          // (head, pair)
+      mw[k] = reinterpret_cast<const uint32_t*>(a.q_mla + (static_cast<int64_t>(q) * kHeads + (j >> 5)) * kDimK +
+                                                kDimV)[j & 31];
+    }
+  }
+
+  // ---- the token's position and slot (no cache write when either is out of range)
   int page = -1;
   if (pos < 0 || pos >= a.max_pages * kPage) {
     if (t == 0) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(pos));
@@ -66,25 +94,23 @@ __global__ void __launch_bounds__(kAppThreads) rope_quantize_append_kernel(const
   const int64_t slot = page >= 0 ? static_cast<int64_t>(page) * kPage + (pos & 63) : -1;
 
   if (t < kRopePairs) {
-    const double theta = pow(static_cast<double>(a.rope_base), -2.0 * t / (2.0 * kRopePairs));
-    const double ang = fmod(static_cast<double>(pos) * theta, 6.283185307179586476925286766559);
-    double s, c;
-    sincos(ang, &s, &c);
-    cs[t] = static_cast<float>(c);
-    sn[t] = static_cast<float>(s);
+    constexpr double kTwoPi = 6.283185307179586476925286766559;
+    const double ang = static_cast<double>(pos) * a.theta[t];
+    const float r = static_cast<float>(ang - rint(ang / kTwoPi) * kTwoPi);
+    float s, c;
+    sincosf(r, &s, &c);
+    cs[t] = c;
+    sn[t] = s;
   }
   if (t < 6) gmax[t] = 0u;
   __syncthreads();
 
   // ---- indexer query: four threads per head, 32 columns each (columns < 64 rotate)
   {
-    const int h = t >> 2, part = t & 3;
-    const uint4* src = reinterpret_cast<const uint4*>(a.idx_q + (static_cast<int64_t>(q) * kHeads + h) * kDimIdx +
-                                                      32 * part);
     float v[32];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 w = src[i];
+      const uint4 w = qw[i];
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -118,7 +144,7 @@ __global__ void __launch_bounds__(kAppThreads) rope_quantize_append_kernel(const
   // ---- indexer key: threads 0..63, one column pair each (pairs < 32 rotate)
   float kx = 0.0f, ky = 0.0f;
   if (t < 64) {
-    const float2 f = bf16x2_to_float2(reinterpret_cast<const uint32_t*>(a.idx_k + static_cast<int64_t>(q) * kDimIdx)[t]);
+    const float2 f = bf16x2_to_float2(kw);
     kx = f.x;
     ky = f.y;
     if (t < kRopePairs) rotate(kx, ky, cs[t], sn[t]);
@@ -134,7 +160,7 @@ __global__ void __launch_bounds__(kAppThreads) rope_quantize_append_kernel(const
   for (int k = 0; k < 2; ++k) {
     const int p = t + kAppThreads * k;
     if (p < kDimK / 2) {
-      const float2 f = bf16x2_to_float2(reinterpret_cast<const uint32_t*>(a.latent + static_cast<int64_t>(q) * kDimK)[p]);
+      const float2 f = bf16x2_to_float2(lw[k]);
       lx[k] = f.x;
       ly[k] = f.y;
       if (p >= kDimV / 2) rotate(lx[k], ly[k], cs[p - kDimV / 2], sn[p - kDimV / 2]);
@@ -149,7 +175,7 @@ __global__ void __launch_bounds__(kAppThreads) rope_quantize_append_kernel(const
       const int j = t + kAppThreads * k;          // (head, pair)
       const int h = j >> 5, i = j & 31;
       uint32_t* w = reinterpret_cast<uint32_t*>(a.q_mla + (static_cast<int64_t>(q) * kHeads + h) * kDimK + kDimV) + i;
-      const float2 f = bf16x2_to_float2(*w);
+      const float2 f = bf16x2_to_float2(mw[k]);
       float x = f.x, y = f.y;
       rotate(x, y, cs[i], sn[i]);
       *w = float2_to_bf16x2(x, y);

@@ -61,7 +61,7 @@ struct AppendArgs {
   const uint16_t* idx_k;    // [Bq, 128]
   const uint16_t* latent;   // [Bq, 576]
   uint16_t* q_mla;          // [Bq, 64, 576] (rope columns rotated in place) or null
-  float rope_base;
+  double theta[32];         // rope_base^(-2i/64), formed on the host in fp64
   uint8_t* q_out;           // [Bq, 64, 128] e4m3
   float* q_scale_out;       // [Bq, 64]
   uint8_t* k_cache;         // [num_pages * 64, 128] e4m3
