@@ -745,39 +745,61 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 // L_{g,s} is split s's normaliser for value group g (columns [128 g, 128 g + 128)): its sum
 // of p for a bf16 cache, and for an fp8 cache the sum of the weights its tensor-core PV
 // actually applied to that group, so that each group is normalised by the weights it used.
-__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+// Two heads per CTA: threads 128 h2 .. + 127 take head 2 blockIdx.y + h2, four consecutive
+// value dims each (warp w of the half owns value group w, the 128 dims that share one
+// normaliser), one 16-byte load per split.
+__global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
   pdl_trigger();
   pdl_wait();   // the partials come from the decode kernel
   const int q = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h = 2 * blockIdx.y + (threadIdx.x >> 7);
+  const int t = threadIdx.x & 127;
+  const int g = t >> 5;                 // value group of dims 4 t .. 4 t + 3
   const int S = a.nsplit;
   const float* ml = a.part_ml + static_cast<int64_t>(q) * S * kHeads * kPartStats;
   float M = -INFINITY;
   for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(s * kHeads + h) * kPartStats]);
-  float Lsum = 0.0f;
-  float Lg[4] = {0.f, 0.f, 0.f, 0.f};
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float Lsum = 0.0f, Lg = 0.0f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = 0; s < S; ++s) {
     const float* st = ml + (s * kHeads + h) * kPartStats;
     const float m = st[0];
     if (m == -INFINITY) continue;
     const float w = exp2f(m - M);
     Lsum += w * st[1];
-    const float* o = a.part_o + ((static_cast<int64_t>(q) * S + s) * kHeads + h) * kDimV;
+    Lg += w * st[2 + g];
+    const float4 o = reinterpret_cast<const float4*>(a.part_o + ((static_cast<int64_t>(q) * S + s) * kHeads + h) * kDimV)[t];
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = Lg > 0.0f ? 1.0f / Lg : 0.0f;
+  const float r[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const int64_t off = (static_cast<int64_t>(q) * kHeads + h) * kDimV + 4 * t;
+  if (a.out_fp32) {
+    float* o = static_cast<float*>(a.out) + off;
+    if ((reinterpret_cast<uintptr_t>(a.out) & 15) == 0) {
+      *reinterpret_cast<float4*>(o) = make_float4(r[0], r[1], r[2], r[3]);
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      Lg[i] += w * st[2 + i];
-      acc[i] += w * o[threadIdx.x + 128 * i];
+      for (int i = 0; i < 4; ++i) o[i] = r[i];
+    }
+  } else {
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.out) + off;
+    if ((reinterpret_cast<uintptr_t>(a.out) & 7) == 0) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(r[0], r[1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(r[2], r[3]);
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(o) = w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = __float2bfloat16_rn(r[i]);
     }
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t off = (static_cast<int64_t>(q) * kHeads + h) * kDimV + threadIdx.x + 128 * i;
-    const float o = Lg[i] > 0.0f ? acc[i] / Lg[i] : 0.0f;
-    if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
-    else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
-  }
-  if (threadIdx.x == 0 && a.lse != nullptr)
+  if (t == 0 && a.lse != nullptr)
     a.lse[static_cast<int64_t>(q) * kHeads + h] = Lsum > 0.0f ? (M + log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
 }
 
@@ -795,7 +817,7 @@ cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cud
   ++*launches;
   if (e != cudaSuccess || a.nsplit == 1) return e;
   ++*launches;
-  return launch_pdl(mla_combine_kernel, dim3(a.Bq, kHeads), dim3(128), 0, stream, a);
+  return launch_pdl(mla_combine_kernel, dim3(a.Bq, kHeads / 2), dim3(256), 0, stream, a);
 }
 
 int mla_tile_keys() { return kMlaTile; }

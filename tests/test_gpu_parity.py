@@ -209,3 +209,24 @@ def test_topk_long_rows_chunked_path():
     for i in range(2):
         check_topk_exact(lo[i], scores[i], vis[i], 2048)
     assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
+
+
+def test_topk_many_queries_mixed_rows():
+    """2400 causal queries over two 4096-token rows (one CTA per query, many waves): rows
+    with ties at the k-th, all-negative scores and planted maxima select exactly."""
+    import torch
+    from tests.gpu_path import GpuCase
+    case = generate(CaseSpec("topk_many", (4096, 4096), top_k=512, n_q=1200, q_tail=True, n_planted=0, seed=41))
+    Bq, L = case["Bq"], 4096
+    rng = np.random.default_rng(42)
+    scores = rng.standard_normal((Bq, L)).astype(np.float32)
+    scores[1::7] = np.round(scores[1::7] * 2) / 2            # few distinct values: ties at the k-th
+    scores[2::7] = -np.abs(scores[2::7])                      # all negative
+    scores[3::7, ::61] += 10.0                                # planted maxima
+    vis = oracle.visible_lengths(case)
+    g = GpuCase(case)
+    lo, ph, err = g.topk(torch.from_numpy(scores).cuda(), 512)
+    assert err == 0
+    for q in range(Bq):
+        check_topk_exact(lo[q], scores[q], vis[q], 512)
+    assert np.array_equal(ph.astype(np.int64), oracle.pagemap(case, lo.astype(np.int64)))
