@@ -17,8 +17,11 @@
 //              (its TMEM lane) applies ReLU, the head weights and the key scale (loaded two
 //              tiles ahead) and writes the fp32 score.
 // Every synchronisation step costs a few hundred nanoseconds, so tiles and units are large
-// enough to keep that cost per byte low. Decode (n_q = 1) loads a row's query once per
-// row; chunked prefill streams groups of up to 4 queries (N = 256) past every key tile.
+// enough to keep that cost per byte low. The work items of a CTA are (row, query group,
+// key tile) in that order, query group outer: a group of up to 4 queries (N = 256) and its
+// head weights stay in place while the row's key tiles stream past it (from L2 after the
+// first group), so decode (one group) and chunked prefill (many) load each query group
+// once per row pass.
 #include "kernels.cuh"
 
 namespace dsa {
@@ -67,18 +70,40 @@ static_assert(IdxCfg<1, 1>::kSmem <= 232448 && IdxCfg<1, 4>::kSmem <= 232448 && 
                   IdxCfg<2, 4>::kSmem <= 232448,
               "shared memory");
 
-// Walks the CTA's contiguous range of global tile ids, yielding (row, tile-in-row) and
-// the row's clamped length. Row bounds and lengths live in registers and are reloaded
-// only when the walk crosses into the next row.
+// Walks the CTA's contiguous range of global work items, yielding (row, query group, key
+// tile) and the row's clamped length: a row's items are its query groups times its key
+// tiles, group-major. Row bounds and lengths live in registers and are reloaded only when
+// the walk crosses into the next row.
+// The longest visible prefix among query group g of row b (out of line: every role's
+// walker calls it once per group).
+template <int QG>
+__device__ __noinline__ int group_vis(const int32_t* q_pos, int n_q, int b, int g, int len) {
+  int v = 0;
+  const int q0 = b * n_q + g * QG;
+  const int nqg = min(QG, n_q - g * QG);
+  for (int j = 0; j < nqg; ++j) v = max(v, query_vis(q_pos, q0 + j, len));
+  return v;
+}
+
+// kVis: also report whether the item is active (a query of its group sees a token of its
+// tile); walkers that only look ahead (key-scale prefetch) take every item as active.
+template <int QG, bool kVis = true>
 struct TileWalker {
   const int32_t* prefix;
   const int32_t* seq_lens;
-  int max_pages;
-  int b, gt, end, base, bound, len;
-  __device__ void init(const IndexerArgs& a, int begin, int stop) {
+  const int32_t* q_pos;
+  int max_pages, tile_tok, n_q;
+  int b, gt, end, base, bound, len, tiles;
+  int vis_b, vis_g, gvis;   // the group whose visible length gvis is cached
+  __device__ void init(const IndexerArgs& a, int tile_tokens, int begin, int stop) {
     prefix = a.tile_prefix;
     seq_lens = a.seq_lens;
+    q_pos = a.q_pos;
+    n_q = a.n_q;
     max_pages = a.max_pages;
+    tile_tok = tile_tokens;
+    vis_b = vis_g = -1;
+    gvis = 0;
     gt = begin;
     end = stop;
     int lo = 0, hi = a.B;  // largest b with prefix[b] <= begin
@@ -90,33 +115,42 @@ struct TileWalker {
     base = prefix[b];
     bound = prefix[b + 1];
     len = row_len(seq_lens, b, max_pages);
+    tiles = (len + tile_tok - 1) / tile_tok;
   }
-  __device__ bool next(int& row, int& tile, int& L) {
+  // `active`: a query of the group sees a token of the tile (every role skips the others)
+  __device__ bool next(int& row, int& group, int& tile, int& L, bool& active) {
     if (gt >= end) return false;
     while (gt >= bound) {
       ++b;
       base = bound;
       bound = prefix[b + 1];
       len = row_len(seq_lens, b, max_pages);
+      tiles = (len + tile_tok - 1) / tile_tok;
     }
     row = b;
-    tile = gt - base;
+    const int i = gt - base;   // < groups * tiles, so tiles >= 1 here
+    if (QG == 1 || n_q <= QG) {   // one group per row: the item is the tile
+      group = 0;
+      tile = i;
+    } else {
+      group = i / tiles;
+      tile = i - group * tiles;
+    }
     L = len;
+    if (kVis) {
+      if (b != vis_b || group != vis_g) {
+        vis_b = b;
+        vis_g = group;
+        gvis = group_vis<QG>(q_pos, n_q, b, group, len);
+      }
+      active = gvis > tile * tile_tok;
+    } else {
+      active = true;
+    }
     ++gt;
     return true;
   }
 };
-
-// A query group contributes to a tile when one of its queries sees a token of it.
-template <int QG>
-__device__ __forceinline__ bool group_active(const IndexerArgs& a, int b, int g, int tok0, int L) {
-  if (a.q_pos == nullptr) return true;
-  const int q0 = b * a.n_q + g * QG;
-  const int nqg = min(QG, a.n_q - g * QG);
-  for (int j = 0; j < nqg; ++j)
-    if (query_vis(a.q_pos, q0 + j, L) > tok0) return true;
-  return false;
-}
 
 template <int KC, int QG>
 __global__ void __launch_bounds__(kIdxThreads, 1)
@@ -183,11 +217,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
   const int t_begin = min(total, static_cast<int>(blockIdx.x) * per);
   const int t_end = min(total, t_begin + per);
-  const int ngroups = (a.n_q + QG - 1) / QG;
 
   if (t_begin < t_end) {
-    TileWalker walk;
-    walk.init(a, t_begin, t_end);
+    TileWalker<QG> walk;
+    walk.init(a, kTileTok, t_begin, t_end);
 
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer (whole warp)
@@ -199,30 +232,33 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
       int it = 0, bit = -1, cur_q0 = -1;
       bool ok = true;
-      auto load_batch = [&](int& n, int& my_b, int& my_t, int& my_L, int& my_page) {
+      // lanes hold the items of a batch; inactive items are marked by my_act = 0
+      auto load_batch = [&](int& n, int& my_b, int& my_g, int& my_t, int& my_act, int& my_page) {
         n = 0;
-        my_b = my_t = my_L = 0;
+        my_b = my_g = my_t = my_act = 0;
+        int my_L = 0;
         for (; n < kBatch; ++n) {
-          int b, t, L;
-          if (!walk.next(b, t, L)) break;
-          if (lane / kPagesPerTile == n) { my_b = b; my_t = t; my_L = L; }
+          int b, g, t, L;
+          bool act;
+          if (!walk.next(b, g, t, L, act)) break;
+          if (lane / kPagesPerTile == n) { my_b = b; my_g = g; my_t = t; my_L = L; my_act = act ? 1 : 0; }
         }
         my_page = -1;
-        if (lane / kPagesPerTile < n) {
+        if (lane / kPagesPerTile < n && my_act) {
           const int p = kPagesPerTile * my_t + (lane % kPagesPerTile);
           if (p * kPage < my_L) my_page = checked_page(a.block_table, my_b, p, a.max_pages, a.num_pages, a.err);
         }
       };
-      int n, my_b, my_t, my_L, my_page;
-      load_batch(n, my_b, my_t, my_L, my_page);
+      int n, my_b, my_g, my_t, my_act, my_page;
+      load_batch(n, my_b, my_g, my_t, my_act, my_page);
       while (ok && n > 0) {
-        int n2, nb, nt, nL, npg;
-        load_batch(n2, nb, nt, nL, npg);
+        int n2, nb, ng, nt, nact, npg;
+        load_batch(n2, nb, ng, nt, nact, npg);
         for (int i = 0; i < n; ++i) {
           const int src = kPagesPerTile * i;
+          if (!__shfl_sync(0xffffffffu, my_act, src)) continue;   // every role skips the item
           const int b = __shfl_sync(0xffffffffu, my_b, src);
-          const int t = __shfl_sync(0xffffffffu, my_t, src);
-          const int L = __shfl_sync(0xffffffffu, my_L, src);
+          const int g = __shfl_sync(0xffffffffu, my_g, src);
           int pages[kPagesPerTile];
 #pragma unroll
           for (int p = 0; p < kPagesPerTile; ++p) pages[p] = __shfl_sync(0xffffffffu, my_page, src + p);
@@ -242,11 +278,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                   tma_load_2d(dst + kc * C::kChunk + p * 8192, &tmap_k, kc * 64, pages[p] * kPage, &a_full[s]);
           }
           ++it;
-          const int tok0 = t * kTileTok;
-          for (int g = 0; g < ngroups; ++g) {
-            if (!group_active<QG>(a, b, g, tok0, L)) continue;
-            const int q0 = b * a.n_q + g * QG;
-            if (q0 == cur_q0) continue;
+          const int q0 = b * a.n_q + g * QG;
+          if (q0 != cur_q0) {
             const int nqg = min(QG, a.n_q - g * QG);
             ++bit;
             const int bs = bit % C::kBSlots;
@@ -261,9 +294,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             }
             cur_q0 = q0;
           }
-          if (!ok) break;
         }
-        n = n2; my_b = nb; my_t = nt; my_L = nL; my_page = npg;
+        n = n2; my_b = nb; my_g = ng; my_t = nt; my_act = nact; my_page = npg;
       }
       if (!ok && lane == 0) {
         record_error(a.err, DSA_ERR_TIMEOUT, 1);
@@ -284,15 +316,15 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 16, 1024);
       int it = 0, bit = -1, cur_q0 = -1, unit = 0;
       bool ok = true;
-      int b, t, L;
-      while (ok && walk.next(b, t, L)) {
+      int b, g, t, L;
+      bool act;
+      while (ok && walk.next(b, g, t, L, act)) {
+        if (!act) continue;
         const int s = it % C::kStages;
         if (!wait_warp(&a_full[s], (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int tok0 = t * kTileTok;
         const uint64_t ad = a_desc0 + static_cast<uint64_t>((s * C::kAStage) >> 4);
-        for (int g = 0; g < ngroups && ok; ++g) {
-          if (!group_active<QG>(a, b, g, tok0, L)) continue;
+        {
           const int q0 = b * a.n_q + g * QG;
           const int nqg = min(QG, a.n_q - g * QG);
           if (q0 != cur_q0) {
@@ -362,14 +394,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
       int unit = 0, cur_q0 = -1, wb = 1;
       bool ok = true;
-      TileWalker w2 = walk, w4 = walk;
+      TileWalker<QG, false> w2, w4;
+      w2.init(a, kTileTok, t_begin, t_end);
       // pages of this thread's tokens in every half of the next tile of walker w (-1 past the end)
-      auto tile_pages = [&](TileWalker& w, int (&p)[H]) {
-        int bb, tt, LL;
+      auto tile_pages = [&](TileWalker<QG, false>& w, int (&p)[H]) {
+        int bb, gg, tt, LL;
+        bool aa;
 #pragma unroll
         for (int h = 0; h < H; ++h) p[h] = -1;
-        if (!w.next(bb, tt, LL)) return;
-        if (a.k_scale == nullptr) return;
+        if (!w.next(bb, gg, tt, LL, aa)) return;
+        if (a.k_scale == nullptr || !aa) return;
 #pragma unroll
         for (int h = 0; h < H; ++h) {
           const int tk = tt * kTileTok + h * 128 + row_in_half;
@@ -391,8 +425,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       w4 = w2;
       tile_pages(w4, pc);             // tile +2
       tile_pages(w4, pd);             // tile +3
-      int b, t, L;
-      while (ok && walk.next(b, t, L)) {
+      int b, g, t, L;
+      bool act;
+      while (ok && walk.next(b, g, t, L, act)) {
         float kscale[H];
 #pragma unroll
         for (int h = 0; h < H; ++h) {
@@ -403,8 +438,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         tile_pages(w4, pd);
         const int tok0 = t * kTileTok;
-        for (int g = 0; g < ngroups && ok; ++g) {
-          if (!group_active<QG>(a, b, g, tok0, L)) continue;
+        if (!act) continue;
+        {
           const int q0 = b * a.n_q + g * QG;
           const int nqg = min(QG, a.n_q - g * QG);
 #pragma unroll
@@ -473,9 +508,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kIdxTmemCols);
 }
 
-// Tile prefix over rows (single CTA) plus validation of lengths and causal positions.
+// Work-item prefix over rows (query groups x key tiles per row; single CTA) plus validation
+// of lengths and causal positions.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q,
-                                                    int max_pages, int tile_tok, int32_t* tile_prefix,
+                                                    int max_pages, int tile_tok, int groups, int32_t* tile_prefix,
                                                     unsigned int* err) {
   __shared__ int warp_sums[32];
   __shared__ int carry;
@@ -493,7 +529,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* seq_lens, con
     if (b < B) {
       const int raw = seq_lens[b];
       if (raw < 0 || raw > max_pages * kPage) record_error(err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(raw));
-      tiles = (row_len(seq_lens, b, max_pages) + tile_tok - 1) / tile_tok;
+      tiles = groups * ((row_len(seq_lens, b, max_pages) + tile_tok - 1) / tile_tok);
     }
     int v = tiles;
 #pragma unroll
@@ -530,11 +566,13 @@ int indexer_tile_tokens(bool fp8, int n_q) {
   return fp8 ? IdxCfg<1, 4>::kTileTok : IdxCfg<2, 4>::kTileTok;
 }
 
+int indexer_query_groups(int n_q) { return n_q == 1 ? 1 : (n_q + 3) / 4; }
+
 cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages, int tile_tok,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches) {
   ++*launches;
   return launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, stream, seq_lens, q_pos, B, n_q, max_pages, tile_tok,
-                    tile_prefix, err);
+                    indexer_query_groups(n_q), tile_prefix, err);
 }
 
 template <int KC, int QG>

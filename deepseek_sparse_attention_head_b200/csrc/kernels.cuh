@@ -19,7 +19,7 @@ struct IndexerArgs {
   const float* k_scale;
   float* scores;
   int64_t L_max;
-  const int32_t* tile_prefix;  // [B+1] exclusive prefix of ceil(len / tile tokens)
+  const int32_t* tile_prefix;  // [B+1] exclusive prefix of query groups x ceil(len / tile tokens)
   unsigned int* err;
 };
 
