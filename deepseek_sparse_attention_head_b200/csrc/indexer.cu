@@ -393,6 +393,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       float* wmine = sW + (warp - 2) * 2 * C::kWPer;   // two buffers of one group's weights per warp
       const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
       int unit = 0, cur_q0 = -1, wb = 1;
+      int qvis[QG];   // visible lengths of the current group's queries (clamped to L_max)
+#pragma unroll
+      for (int j = 0; j < QG; ++j) qvis[j] = 0;
       bool ok = true;
       TileWalker<QG, false> w2, w4;
       w2.init(a, kTileTok, t_begin, t_end);
@@ -442,7 +445,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         {
           const int q0 = b * a.n_q + g * QG;
           const int nqg = min(QG, a.n_q - g * QG);
-#pragma unroll
+#pragma unroll 1
           for (int u = 0; u < kUnitsPerTile; ++u, ++unit) {
             if ((unit & 1) != eg) continue;
             if (q0 != cur_q0) {
@@ -452,6 +455,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 float w = a.head_w[static_cast<int64_t>(q0) * kHeads + i];
                 if (a.q_scale != nullptr) w *= a.q_scale[static_cast<int64_t>(q0) * kHeads + i];
                 wmine[wb * C::kWPer + i] = w;
+              }
+#pragma unroll
+              for (int j = 0; j < QG; ++j) {
+                int v = j < nqg ? query_vis(a.q_pos, q0 + j, L) : 0;
+                qvis[j] = v > a.L_max ? static_cast<int>(a.L_max) : v;
               }
               __syncwarp();
               cur_q0 = q0;
@@ -466,6 +474,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             for (int hh = 0; hh < UH; ++hh) {
               const int h2 = u * UH + hh;
               const int tok = tok0 + h2 * 128 + row_in_half;
+#pragma unroll 1
               for (int j = 0; j < nqg; ++j) {
                 float acc[64];
                 tmem_ld64(lane_addr + static_cast<uint32_t>(ab * unit_cols + hh * acc_cols + j * kHeads), acc);
@@ -482,10 +491,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 }
                 const float sc =
                     ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-                const int q = q0 + j;
-                int vis = query_vis(a.q_pos, q, L);
-                if (vis > a.L_max) vis = static_cast<int>(a.L_max);
-                if (tok < vis) a.scores[static_cast<int64_t>(q) * a.L_max + tok] = sc * kscale[h2];
+                int vis = qvis[0];
+#pragma unroll
+                for (int jj = 1; jj < QG; ++jj)
+                  if (jj == j) vis = qvis[jj];
+                if (tok < vis) a.scores[static_cast<int64_t>(q0 + j) * a.L_max + tok] = sc * kscale[h2];
               }
             }
             tc_fence_before();
