@@ -479,15 +479,24 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 float acc[64];
                 tmem_ld64(lane_addr + static_cast<uint32_t>(ab * unit_cols + hh * acc_cols + j * kHeads), acc);
                 const float4* wq = reinterpret_cast<const float4*>(wmine + wb * C::kWPer + j * kHeads);
-                float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent chains
+                // ReLU per head, then head pairs through packed fp32x2 FMAs: eight independent
+                // chains (head h feeds chain 4 (h / 4 & 1) + h % 4), as four packed registers
+                uint64_t pp[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int h4 = 0; h4 < 16; ++h4) {
                   const float4 w = wq[h4];
-                  float* pp = part + 4 * (h4 & 1);
-                  pp[0] = fmaf(w.x, fmaxf(acc[4 * h4 + 0], 0.0f), pp[0]);
-                  pp[1] = fmaf(w.y, fmaxf(acc[4 * h4 + 1], 0.0f), pp[1]);
-                  pp[2] = fmaf(w.z, fmaxf(acc[4 * h4 + 2], 0.0f), pp[2]);
-                  pp[3] = fmaf(w.w, fmaxf(acc[4 * h4 + 3], 0.0f), pp[3]);
+                  uint64_t* c = pp + 2 * (h4 & 1);
+                  c[0] = fma_f32x2(pack_f32x2(w.x, w.y),
+                                   pack_f32x2(fmaxf(acc[4 * h4 + 0], 0.0f), fmaxf(acc[4 * h4 + 1], 0.0f)), c[0]);
+                  c[1] = fma_f32x2(pack_f32x2(w.z, w.w),
+                                   pack_f32x2(fmaxf(acc[4 * h4 + 2], 0.0f), fmaxf(acc[4 * h4 + 3], 0.0f)), c[1]);
+                }
+                float part[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f = unpack_f32x2(pp[i]);
+                  part[2 * i] = f.x;
+                  part[2 * i + 1] = f.y;
                 }
                 const float sc =
                     ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
