@@ -187,14 +187,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  if (ntiles > 0 && tid == 0) tma_prefetch_map(&tmap_q);
+
+  pdl_trigger();
+  // The slot list comes from top-k, and any earlier kernel on the stream may still be
+  // writing the queries (the cache append rotates their rope columns in place): nothing
+  // from global memory is read before this wait.
+  pdl_wait();
   if (ntiles > 0 && tid == 0) {
-    tma_prefetch_map(&tmap_q);
     mbar_arrive_expect_tx(q_full, 9u * 8192u);
     for (int c = 0; c < 9; ++c) tma_load_2d(sQ + c * 8192, &tmap_q, c * 64, q * kHeads, q_full);
   }
-
-  pdl_trigger();
-  pdl_wait();   // the slot list comes from top-k
 
   // the split's slot list, staged once when it fits (invalid entries become -1)
   const bool list_in_smem = ntiles * kMlaTile <= kIdxListCap;

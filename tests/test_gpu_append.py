@@ -151,3 +151,69 @@ def test_position_outside_the_table_reports_and_writes_nothing():
     assert set(changed.tolist()) <= {slot0}
     changed_kv = np.nonzero((kv_cache.cpu().numpy() != case["kv_cache"]).any(axis=1))[0]
     assert set(changed_kv.tolist()) <= {slot0} and slot0 in changed_kv.tolist()
+
+
+def test_decode_right_after_append_sees_the_rotated_queries():
+    """mla_sparse_decode replayed from one CUDA graph directly behind dsa_rope_quantize_append
+    (programmatic dependent launch lets the second kernel start while the first runs) reads
+    the queries only after the append has rotated them: its output equals that of the same
+    two calls separated by a device synchronisation, bit for bit."""
+    import torch
+    import deepseek_sparse_attention_head_b200 as dsa
+    case = generate(CaseSpec("app_then_mla", (3000, 1500, 4100, 2222) * 16, top_k=512, kv_dtype="fp8", seed=87))
+    new = new_token_inputs(case, seed=9)
+    t = to_torch(case, "cuda")
+    Bq = case["Bq"]
+    vis = oracle.visible_lengths(case)
+    logical = np.full((Bq, 512), -1, dtype=np.int64)
+    for q in range(Bq):
+        n = min(512, int(vis[q]))
+        logical[q, :n] = np.arange(int(vis[q]) - n, int(vis[q]))    # the newest tokens, the new one included
+    phys = torch.from_numpy(oracle.pagemap(case, logical).astype(np.int32)).cuda()
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).view(torch.int16).view(torch.bfloat16).cuda()
+    paging = dsa.Paging(t["seq_lens"], t["block_table"], case["num_pages"], case["n_q"], t["q_pos"])
+    q0, iq, ik, lat = bf(new["q_mla"]), bf(new["idx_q"]), bf(new["idx_k"]), bf(new["latent"])
+    q_mla = q0.clone()
+    k_cache, k_scale = t["k_cache"].view(torch.uint8).clone(), t["k_scale"].clone()
+    kv_cache, kv_scale = t["kv_cache"].clone(), t["kv_scale"].clone()
+    q_out = torch.empty(Bq, 64, 128, dtype=torch.uint8, device="cuda")
+    q_sc = torch.empty(Bq, 64, dtype=torch.float32, device="cuda")
+    out = torch.empty((Bq, 64, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(Bq, 64, dtype=torch.float32, device="cuda")
+    ws = dsa.alloc_workspace(dsa.mla_workspace_size(Bq, 512))
+
+    def reset():
+        q_mla.copy_(q0)
+        k_cache.copy_(t["k_cache"].view(torch.uint8))
+        k_scale.copy_(t["k_scale"])
+        kv_cache.copy_(t["kv_cache"])
+        kv_scale.copy_(t["kv_scale"])
+        out.fill_(float("nan"))
+        torch.cuda.synchronize()
+
+    def append():
+        dsa.dsa_rope_quantize_append(paging, iq, ik, lat, q_mla, q_out, q_sc, k_cache, k_scale, kv_cache, kv_scale)
+
+    def decode():
+        dsa.mla_sparse_decode(q_mla, kv_cache, kv_scale, phys, case["softmax_scale"], out, lse, ws)
+
+    reset()
+    append()
+    torch.cuda.synchronize()
+    decode()
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_error(ws) == 0
+    want = (out.view(torch.int16).cpu().numpy(), lse.cpu().numpy())
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            append()
+            decode()
+    for _ in range(5):
+        reset()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert dsa.dsa_get_error(ws) == 0
+        assert np.array_equal(out.view(torch.int16).cpu().numpy(), want[0])
+        assert np.array_equal(lse.cpu().numpy(), want[1])
