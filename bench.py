@@ -253,6 +253,127 @@ def time_stage(call, reps, nbytes, stream, flush):
             f"the call alone, L2 flushed before each ({nbytes / 1e6:.1f} MB < L2), mean of {reps}")
 
 
+def e2e_serial(t, in_keys, pin, host_out, host_lse, out, lse, step, stream, flush, n, use_graph, world):
+    """Device ms of n steps, each copy-in, layer call and copy-out in turn on one stream and
+    timed alone after an L2 flush (for workloads that fit in L2)."""
+
+    def body():
+        for k in in_keys:
+            t[k].copy_(pin[k], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+
+    g = None
+    if use_graph:
+        with torch.cuda.stream(stream):
+            body()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            body()
+        stream.synchronize()
+    call = g.replay if g is not None else body
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = timed_flushed(call, n, stream, flush)
+    torch.cuda.synchronize()
+    del g
+    how = "serial steps from one CUDA graph each (copies included), L2 flushed before each" if use_graph else \
+        "serial eager steps (copies included), L2 flushed before each"
+    return ms, how
+
+
+def e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, stream, n, use_graph, world):
+    """Device ms from the first copy-in to the last copy-out of n steps over two buffer sets,
+    as a serving loop overlaps them: while step k computes on set k % 2, step k+1's inputs
+    are copied into the other set (its own stream) and step k-1's output and lse are copied
+    out of it (a third stream). One pipeline stage (copy-in, layer, copy-out, forked and
+    joined) is one CUDA graph per set parity. The first stage's copy-out and the last
+    stage's copy-in move bytes no step uses: n + 1 copies each way for n steps."""
+    K = case["top_k"]
+    sets = []
+    for si in range(2):
+        dev = {k: (t[k] if si == 0 else t[k].clone()) for k in in_keys}
+        pg = dsa.Paging(dev["seq_lens"], dev["block_table"], case["num_pages"], case["n_q"], t["q_pos"])
+        sets.append((dev, pg, out if si == 0 else torch.empty_like(out), lse if si == 0 else torch.empty_like(lse)))
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def copy_in(si):
+        with torch.cuda.stream(cin):
+            for k in in_keys:
+                sets[si][0][k].copy_(pin[k], non_blocking=True)
+
+    def copy_out(si):
+        with torch.cuda.stream(cout):
+            host_out.copy_(sets[si][2], non_blocking=True)
+            host_lse.copy_(sets[si][3], non_blocking=True)
+
+    def stage(si):
+        """Step on set si; the other set's inputs in and outputs out meanwhile."""
+        other = 1 - si
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        cin.wait_event(fork)
+        cout.wait_event(fork)
+        copy_in(other)
+        copy_out(other)
+        dev, pg, o, l = sets[si]
+        with torch.cuda.stream(stream):
+            dsa.dsa_decode_layer(pg, dev["q_idx"], dev["q_idx_scale"], dev["head_w"], t["k_cache"], t["k_scale"],
+                                 dev["q_mla"], t["kv_cache"], t["kv_scale"], K, case["softmax_scale"], o, ws, lse=l,
+                                 stream=stream)
+        j_in, j_out = torch.cuda.Event(), torch.cuda.Event()
+        j_in.record(cin)
+        j_out.record(cout)
+        stream.wait_event(j_in)
+        stream.wait_event(j_out)
+
+    graphs = [None, None]
+    if use_graph:
+        for si in range(2):
+            stage(si)
+            torch.cuda.synchronize()
+            graphs[si] = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graphs[si], stream=stream):
+                stage(si)
+            torch.cuda.synchronize()
+
+    def run(count):
+        copy_in(0)
+        ready = torch.cuda.Event()
+        ready.record(cin)
+        stream.wait_event(ready)
+        for k in range(count):
+            with torch.cuda.stream(stream):
+                if graphs[k % 2] is not None:
+                    graphs[k % 2].replay()
+                else:
+                    stage(k % 2)
+        last = torch.cuda.Event()
+        last.record(stream)
+        cout.wait_event(last)
+        copy_out((count - 1) % 2)
+
+    run(4)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cin)
+    run(n)
+    e1.record(cout)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del graphs
+    how = ("pipelined over two buffer sets: copy-in of the next step and copy-out of the previous one overlap "
+           "each step, " + ("one CUDA graph per stage" if use_graph else "eager launches"))
+    return ms, how
+
+
 def run_ours(args, world, rank, local):
     import deepseek_sparse_attention_head_b200 as dsa
 
@@ -350,49 +471,21 @@ def run_ours(args, world, rank, local):
     if dsa.dsa_get_error(ws_m, stream) != 0:
         raise RuntimeError("device error in the MLA timing calls")
 
-    # ---- end to end through the public API with host buffers
-    pin = {k: t[k].cpu().pin_memory() for k in ("q_idx", "q_idx_scale", "head_w", "q_mla", "seq_lens",
-                                                   "block_table") if t[k] is not None}
+    # ---- end to end through the public API with host buffers: every step copies its
+    # query-side inputs in from pinned host memory and its output and lse back out
+    in_keys = [k for k in ("q_idx", "q_idx_scale", "head_w", "q_mla", "seq_lens", "block_table") if t[k] is not None]
+    pin = {k: t[k].cpu().pin_memory() for k in in_keys}
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
     d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
     n_e2e = max(10, args.e2e_steps)
-
-    def e2e_body():
-        for k, v in pin.items():
-            t[k].copy_(v, non_blocking=True)
-        step()
-        host_out.copy_(out, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
-
-    # the whole step, host copies included, replayed from one CUDA graph (as a serving loop
-    # would run it); eager launches when graphs are off
-    e2e_graph = None
-    if graph is not None:
-        with torch.cuda.stream(stream):
-            e2e_body()
-        stream.synchronize()
-        e2e_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(e2e_graph, stream=stream):
-            e2e_body()
-        stream.synchronize()
-
-    def e2e_step():
-        if e2e_graph is not None:
-            e2e_graph.replay()
-        else:
-            e2e_body()
-
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            e2e_step()
-    barrier(world)
-    torch.cuda.synchronize()
     if inputs_exceed_l2:
-        e2e_local = timed_back_to_back(e2e_step, n_e2e, stream)
+        e2e_local, e2e_how = e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, stream,
+                                           n_e2e, graph is not None, world)
     else:
-        e2e_local = timed_flushed(e2e_step, n_e2e, stream, flush)
+        e2e_local, e2e_how = e2e_serial(t, in_keys, pin, host_out, host_lse, out, lse, step, stream, flush, n_e2e,
+                                        graph is not None, world)
     e2e_ms = max_over_ranks(e2e_local, world)
 
     hbm_peak, bf16_peak, peak_kind = measured_peaks()
@@ -468,8 +561,7 @@ def run_ours(args, world, rank, local):
         "roofline": roofline,
         "roofline_other_kernel": other,
         "e2e": {"value": world * n_e2e / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": n_e2e,
-                "launch": "cuda_graph (copies included)" if e2e_graph is not None else "eager"},
+                "d2h_bytes_per_step": d2h, "steps": n_e2e, "launch": e2e_how},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
@@ -477,8 +569,6 @@ def run_ours(args, world, rank, local):
         result["fp8_tensor_peak"] = {"tflops": fp8_peak, "how": fp8_how}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(case, budget_s=20.0)
-    if e2e_graph is not None:
-        del e2e_graph
     if graph is not None:
         del graph
     return result
