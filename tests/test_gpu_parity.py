@@ -29,6 +29,15 @@ SMALL = {
     "packed_fp8": CaseSpec("packed_fp8", (37, 64, 200, 1, 129), top_k=64, kv_dtype="fp8r", seed=40),
     "mtp_bf16": CaseSpec("mtp_bf16", (129, 640), top_k=64, n_q=4, q_tail=True, idx_dtype="bf16", kv_dtype="bf16",
                          out_dtype="fp32", n_planted=0, seed=39),
+    # chunked prefill with causal queries spread from the first token to the shortest row's
+    # end (nine queries: two full query groups and a partial one; the same positions in
+    # every row), so that many (query group, key tile) work items of the indexer see no
+    # token, in the longer rows whole runs of tiles, and are skipped by every role
+    "prefill_spread": CaseSpec("prefill_spread", (5000, 3000, 1200), top_k=256, n_q=9,
+                               q_pos=(0, 100, 255, 256, 511, 700, 900, 1100, 1199), n_planted=0, seed=41),
+    "prefill_spread_bf16": CaseSpec("prefill_spread_bf16", (700, 2100), top_k=128, n_q=5,
+                                    q_pos=(3, 255, 256, 511, 699),
+                                    idx_dtype="bf16", kv_dtype="bf16", out_dtype="fp32", n_planted=0, seed=42),
 }
 FULL = ["cfg0", "cfg1"]
 
