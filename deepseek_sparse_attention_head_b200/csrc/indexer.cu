@@ -232,6 +232,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
       int it = 0, bit = -1, cur_q0 = -1;
       bool ok = true;
+      // With one query group per row every key page is read once: it goes to L2 as first to
+      // be evicted, so that the streamed keys do not displace the scores, which the top-k
+      // reads next. With several groups the row's keys are read again from L2.
+      const bool keys_once = a.n_q <= QG;
+      const uint64_t evict_first = l2_evict_first_policy();
       // lanes hold the items of a batch; inactive items are marked by my_act = 0
       auto load_batch = [&](int& n, int& my_b, int& my_g, int& my_t, int& my_act, int& my_page) {
         n = 0;
@@ -274,8 +279,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             for (int p = 0; p < kPagesPerTile; ++p)
               if (pages[p] >= 0)
 #pragma unroll
-                for (int kc = 0; kc < KC; ++kc)
-                  tma_load_2d(dst + kc * C::kChunk + p * 8192, &tmap_k, kc * 64, pages[p] * kPage, &a_full[s]);
+                for (int kc = 0; kc < KC; ++kc) {
+                  if (keys_once)
+                    tma_load_2d_hint(dst + kc * C::kChunk + p * 8192, &tmap_k, kc * 64, pages[p] * kPage, &a_full[s],
+                                     evict_first);
+                  else
+                    tma_load_2d(dst + kc * C::kChunk + p * 8192, &tmap_k, kc * 64, pages[p] * kPage, &a_full[s]);
+                }
           }
           ++it;
           const int q0 = b * a.n_q + g * QG;
