@@ -222,6 +222,7 @@ dsa_status run_topk(const dsa_paging* pg, const float* scores, int64_t L_max, in
   a.physical = physical;
   a.err = err_word(ws);
   a.chunks = lay.tk_chunks;
+  a.pair = lay.tk_chunks <= 1 ? topk_pairs(static_cast<int>(Bq), L_max, device_sms()) : 0;
   a.cand_cap = topk_candidate_capacity();
   a.g_cnt = a.g_rmax = a.g_thr = a.g_key = nullptr;
   a.g_idx = nullptr;

@@ -39,6 +39,7 @@ struct TopkArgs {
   // long-row gather (chunks > 1): per-query candidate count, largest key - threshold,
   // threshold, and candidate buffers [Bq, cand_cap]; counts and maxima start at zero
   int chunks;
+  int pair;   // 1: each row over a cluster of two CTAs (chunks == 1 only)
   int cand_cap;
   uint32_t* g_cnt;
   uint32_t* g_rmax;
@@ -130,6 +131,27 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// launch_pdl for a grid of thread-block clusters of `cluster_x` CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                      cudaStream_t stream, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Each returns the launch error (cudaSuccess when queued) and adds the number of
 // kernels it queued to *launches.
 // Tokens per indexer tile for this cache type and query count (the plan's tile unit).
@@ -140,6 +162,8 @@ cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMa
                            int grid, cudaStream_t stream, int* launches);
 // Chunks per row of the long-row top-k (1 = one CTA per query) and its candidate capacity.
 int topk_chunks(int Bq, int64_t L_max, int sms);
+// 1 when each row's gather is split over a cluster of two CTAs (all pairs in one wave).
+int topk_pairs(int Bq, int64_t L_max, int sms);
 int topk_candidate_capacity();
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches);
 cudaError_t launch_pagemap(int n_q, int top_k, int64_t total, const int32_t* block_table, int max_pages,

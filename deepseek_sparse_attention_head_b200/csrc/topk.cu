@@ -18,6 +18,8 @@
 // chunks, one CTA each, into a per-row candidate buffer in the workspace; a second
 // kernel then runs step 3 per row.
 // A query that sees no more than top_k tokens takes all of them (the dense path).
+#include <cooperative_groups.h>
+
 #include "kernels.cuh"
 
 namespace dsa {
@@ -537,6 +539,51 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
   select_whole_row(sm, a, rw);
 }
 
+// Rows gathered by a cluster of two CTAs (query = cluster index): both derive the same
+// threshold, each gathers half of the row straight into the first CTA's candidate buffer
+// (distributed shared memory, its counters and atomics), and after the cluster barrier the
+// first CTA selects and emits. One SM pulls a row at ~16 B/cycle, so two halve the gather.
+// Every branch taken before the barriers depends only on the row, the same in both CTAs.
+__global__ void __launch_bounds__(kTopkThreads) topk_pair_kernel(const TopkArgs a) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned rank = cluster.block_rank();
+  pdl_trigger();
+  pdl_wait();   // scores come from the indexer
+  const TopkRow rw = topk_row(a, static_cast<int>(blockIdx.x >> 1));
+  if (rw.vis <= rw.K) {
+    if (rank == 0) topk_dense(a, rw);
+    return;
+  }
+  if ((reinterpret_cast<uintptr_t>(rw.row) & 15) != 0) {
+    if (rank == 0) select_whole_row(sm, a, rw);
+    return;
+  }
+  const int mid = min(rw.vis, ((rw.vis >> 1) + 15) & ~15);   // a multiple of 4: 16-byte loads stay aligned
+  const int lo = rank == 0 ? 0 : mid;
+  const int hi = rank == 0 ? mid : rw.vis;
+  float4 first[kGatherU / 4];
+  gather_load(rw.row, lo, hi, first);   // in flight while the threshold is derived
+  const uint32_t thr = row_threshold_small(sm, rw.row, rw.vis, rw.K);
+  if (threadIdx.x == 0) {
+    sm.n_cand = 0;
+    sm.rmax = 0;
+  }
+  cluster.sync();   // the first CTA's counters are zero before either half adds to them
+  TopkSmem& dst = rank == 0 ? sm : *cluster.map_shared_rank(&sm, 0);
+  gather_range(rw.row, lo, hi, thr, &dst.n_cand, dst.cand_key, dst.cand_idx, kCand, &dst.rmax, first);
+  cluster.sync();   // both halves' candidates are in the first CTA's buffer
+  if (rank != 0) return;
+  const uint32_t n_c = sm.n_cand;
+  if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand)) {
+    select_and_emit(sm, a, rw, n_c, thr, sm.rmax);
+    return;
+  }
+  select_whole_row(sm, a, rw);
+}
+
 // Long rows, part 1: grid (chunks, queries). Each CTA derives the row's threshold (the same
 // in every chunk CTA) and gathers the candidates of its 16K-key chunk into the row's
 // global candidate buffer.
@@ -622,10 +669,21 @@ int topk_chunks(int Bq, int64_t L_max, int sms) {
   return c < 2 ? 1 : static_cast<int>(c);
 }
 
+int topk_pairs(int Bq, int64_t L_max, int sms) {
+  // every pair resident at once (one 1024-thread CTA per SM), rows long enough to split
+  return Bq > 0 && sms > 0 && 2LL * Bq <= sms && L_max >= 32768 ? 1 : 0;
+}
+
 int topk_candidate_capacity() { return kCand; }
 
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches) {
   const int smem = static_cast<int>(sizeof(TopkSmem));
+  if (a.chunks <= 1 && a.pair) {
+    cudaError_t e = set_smem_once<topk_pair_kernel>(smem);
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    return launch_pdl_cluster(topk_pair_kernel, dim3(2 * Bq), dim3(kTopkThreads), smem, stream, 2u, a);
+  }
   if (a.chunks <= 1) {
     cudaError_t e = set_smem_once<topk_pagemap_kernel>(smem);
     if (e != cudaSuccess) return e;

@@ -239,3 +239,22 @@ def test_topk_many_queries_mixed_rows():
     for q in range(Bq):
         check_topk_exact(lo[q], scores[q], vis[q], 512)
     assert np.array_equal(ph.astype(np.int64), oracle.pagemap(case, lo.astype(np.int64)))
+
+
+def test_topk_rows_over_two_ctas():
+    """Rows of 40K keys for a few queries take the layout where a cluster of two CTAs
+    gathers each row's halves into one candidate buffer: a constant row (the buffer
+    overflows and the first CTA falls back to the whole-row select after the cluster
+    barrier), few distinct values (ties at the k-th), a near-constant row, all-negative
+    scores, a random row with an odd visible length, and a row shorter than top_k."""
+    rng = np.random.default_rng(7)
+    L = 40000
+    rows = [np.full(L, 0.5), rng.choice([0.25, 0.5, 1.0], size=L), rng.standard_normal(L) * 1e-3 + 7.0,
+            -np.abs(rng.standard_normal(L)), rng.standard_normal(L), rng.standard_normal(L)]
+    scores = np.stack(rows).astype(np.float32)
+    vis = np.array([L, L - 5, 39000, L, 33333, 1500])
+    case, lo, ph, err = _topk_on_scores(scores, vis, 2048)
+    assert err == 0
+    for i in range(len(rows)):
+        check_topk_exact(lo[i], scores[i], vis[i], 2048)
+    assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
