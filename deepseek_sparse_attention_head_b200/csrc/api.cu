@@ -267,6 +267,7 @@ dsa_status run_mla(int Bq, const void* q, const void* kv, dsa_dtype kv_dtype, co
   a.err = err_word(ws);
   a.wait_limit = g_test_wait_limit > 0 ? g_test_wait_limit : kWaitLimitCycles;
   a.stall = g_test_stall;
+  a.pair = a.nsplit == 2 ? 1 : 0;
   const int kvf = kv_dtype == DSA_FP8_E4M3 ? kKvFp8 : kv_dtype == DSA_FP8_E4M3_ROPE_BF16 ? kKvFp8Packed : kKvBf16;
   return cuda_status(launch_mla(kvf, tq, a, st, &g_launches));
 }

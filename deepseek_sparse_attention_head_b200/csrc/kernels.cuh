@@ -96,6 +96,7 @@ struct MlaArgs {
   unsigned int* err;
   long long wait_limit; // bound of every wait, in SM cycles (kWaitLimitCycles unless a test shortens it)
   int stall;            // test hook: the softmax warps wait on a barrier nothing arrives on
+  int pair;             // nsplit == 2 launched as clusters of two: the splits merge in the kernel
 };
 
 // Raises kernel K's dynamic shared-memory limit once per device (a host-side cost that

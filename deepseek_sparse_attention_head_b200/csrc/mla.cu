@@ -26,6 +26,7 @@
 // Q is staged once per CTA and rescaled per head by a power of two into fp16. With
 // a bf16 cache the same pipeline runs in bf16 without any rescaling.
 // Splits write (m, l, o) partials that mla_combine_kernel merges by log-sum-exp.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -139,6 +140,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
   float* sAlpha = sCq + 64;
   float* sOutScale = sCq + 128;
   int32_t* sIdxList = reinterpret_cast<int32_t*>(smem + kOffIdxList);
+  // Pair merge (a.pair), over the slot list once the tile loop is over: per head the split's
+  // running max (log2 units) and sum of p, then the merge factors; kPairGood: the split's O is valid.
+  float* sPair = reinterpret_cast<float*>(smem + kOffIdxList);
+  constexpr int kPairM = 0, kPairL = 64, kPairMul = 128, kPairInvL = 192, kPairOn = 256, kPairGood = 320;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
   uint64_t* q_full = bars + 0;
   uint64_t* q_ready = bars + 1;
@@ -435,7 +440,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const float l = l_run;
         const float oscale = exp2i(e_ref == kNoExp ? 0 : e_ref);
         sOutScale[h] = split_out ? oscale : (l > 0.0f ? oscale / l : 0.0f);
-        if (split_out) {
+        if (a.pair) {
+          sPair[kPairM + h] = l > 0.0f ? m_run : -INFINITY;
+          sPair[kPairL + h] = l;
+        } else if (split_out) {
           float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kPartStats;
           ml[0] = l > 0.0f ? m_run : -INFINITY;
 #pragma unroll
@@ -452,8 +460,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     if (!(good && got) && lane == 0) *abort_flag = 1;
     // O is final and the scales are published: the loaders join the readout
     good = bar_and(kEpiBar, kEpiThreads, good && got) != 0;
-    if (good) write_out(0);
-    if (!good && a.nsplit > 1 && is_sm) {
+    if (good && !a.pair) write_out(0);
+    if (a.pair) {
+      if (!good && is_sm) {
+        sPair[kPairM + h] = -INFINITY;
+        sPair[kPairL + h] = 0.0f;
+      }
+      if (tid == 0) sPair[kPairGood] = good ? 1.0f : 0.0f;
+    } else if (!good && a.nsplit > 1 && is_sm) {
       // an empty partial, so the combine skips this split instead of reading stale data
       float* ml = a.part_ml + ((static_cast<int64_t>(q) * a.nsplit + split) * kHeads + h) * kPartStats;
       ml[0] = -INFINITY;
@@ -709,10 +723,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     __syncwarp();
     // the output epilogue with the softmax warps (they publish the per-head scales first)
-    if (bar_and(kEpiBar, kEpiThreads, good) != 0) write_out(warp <= kLoadWarp0 + 3 ? 1 : 2);
+    if (bar_and(kEpiBar, kEpiThreads, good) != 0 && !a.pair) write_out(warp <= kLoadWarp0 + 3 ? 1 : 2);
   }
 
-  if (ntiles == 0) {
+  if (ntiles == 0 && a.pair) {
+    // nothing selected in this split: an empty one for the merge (no O is read from TMEM)
+    if (tid < kHeads) {
+      sPair[kPairM + tid] = -INFINITY;
+      sPair[kPairL + tid] = 0.0f;
+      sOutScale[tid] = 0.0f;
+    }
+    if (tid == 0) sPair[kPairGood] = 1.0f;
+  } else if (ntiles == 0) {
     // nothing selected: zero output (or an empty partial)
     const bool split_out = a.nsplit > 1;
     for (int i = tid; i < kHeads * kDimV; i += kMlaThreads) {
@@ -733,6 +755,81 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         for (int i = 1; i < kPartStats; ++i) ml[i] = 0.0f;
       } else if (a.lse != nullptr) {
         a.lse[static_cast<int64_t>(q) * kHeads + tid] = -INFINITY;
+      }
+    }
+  }
+
+  if (a.pair) {
+    // ---------------------------------------------------------------- merge of the two splits
+    // Split s owns heads 32 s .. 32 s + 31. After the first cluster barrier each CTA reads the
+    // other's (m, l), both derive the same weights, and each writes the other's head half of
+    // its O (times its weight) into the other's first tile buffer, now free; after the
+    // second barrier each normalises its own half. Every thread of both CTAs reaches both
+    // barriers: all roles above end here, and every wait before is bounded.
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int peer = split ^ 1;
+    tc_fence_before();
+    cluster.sync();
+    tc_fence_after();
+    if (tid < kHeads) {
+      const float* pp = cluster.map_shared_rank(sPair, static_cast<unsigned>(peer));
+      const bool peer_good = pp[kPairGood] != 0.0f;
+      const float ms = sPair[kPairM + tid], ls = sPair[kPairL + tid];
+      const float mp = peer_good ? pp[kPairM + tid] : -INFINITY;
+      const float lp = peer_good ? pp[kPairL + tid] : 0.0f;
+      const float M = fmaxf(ms, mp);
+      const float ws = ls > 0.0f ? exp2f(ms - M) : 0.0f;
+      const float wp = lp > 0.0f ? exp2f(mp - M) : 0.0f;
+      const float L = ws * ls + wp * lp;
+      sPair[kPairMul + tid] = ws * sOutScale[tid];
+      sPair[kPairInvL + tid] = L > 0.0f ? 1.0f / L : 0.0f;
+      sPair[kPairOn + tid] = wp > 0.0f ? 1.0f : 0.0f;
+      if ((tid >> 5) == split && a.lse != nullptr)
+        a.lse[static_cast<int64_t>(q) * kHeads + tid] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+    // a split with nothing selected sends nothing (its weight is 0) but writes its own heads
+    const bool epi = (warp < 4 || warp >= kLoadWarp0) && sPair[kPairGood] != 0.0f;
+    const bool send = epi && ntiles > 0;
+    const int part = warp < 4 ? 0 : (warp <= kLoadWarp0 + 3 ? 1 : 2);   // three warps per lane quadrant
+    const int quad = warp & 3;
+    const uint32_t lb = static_cast<uint32_t>(quad * 32) << 16;
+    float* recv = reinterpret_cast<float*>(sKV);                        // [32 heads][512 dims]
+    if (send) {
+      float* precv = cluster.map_shared_rank(recv, static_cast<unsigned>(peer));
+#pragma unroll 1
+      for (int d = part; d < 4; d += 3) {
+        const int dim = d * 128 + quad * 32 + lane;
+        float v[32];
+        tmem_ld32(tmem + kTmemO + lb + d * 64 + peer * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float mul = sPair[kPairMul + peer * 32 + i];
+          precv[i * kDimV + dim] = mul != 0.0f ? v[i] * mul : 0.0f;
+        }
+      }
+    }
+    tc_fence_before();
+    cluster.sync();
+    tc_fence_after();
+    if (epi) {
+#pragma unroll 1
+      for (int d = part; d < 4; d += 3) {
+        const int dim = d * 128 + quad * 32 + lane;
+        float v[32];
+        tmem_ld32(tmem + kTmemO + lb + d * 64 + split * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int hh = split * 32 + i;
+          const float mul = sPair[kPairMul + hh];
+          const float own = mul != 0.0f ? v[i] * mul : 0.0f;
+          const float other = sPair[kPairOn + hh] != 0.0f ? recv[i * kDimV + dim] : 0.0f;
+          const float o = (own + other) * sPair[kPairInvL + hh];
+          const int64_t off = (static_cast<int64_t>(q) * kHeads + hh) * kDimV + dim;
+          if (a.out_fp32) static_cast<float*>(a.out)[off] = o;
+          else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(o);
+        }
       }
     }
   }
@@ -810,6 +907,9 @@ template <int KVF>
 static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStream_t stream) {
   cudaError_t e = set_smem_once<mla_decode_kernel<KVF>>(kMlaSmem);
   if (e != cudaSuccess) return e;
+  if (a.pair)
+    return launch_pdl_cluster(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, 2u,
+                              tq, a);
   return launch_pdl(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
 }
 
@@ -818,7 +918,7 @@ cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cud
                   : kvf == kKvFp8     ? launch_mla_t<kKvFp8>(tmap_q, a, stream)
                                       : launch_mla_t<kKvBf16>(tmap_q, a, stream);
   ++*launches;
-  if (e != cudaSuccess || a.nsplit == 1) return e;
+  if (e != cudaSuccess || a.nsplit == 1 || a.pair) return e;
   ++*launches;
   return launch_pdl(mla_combine_kernel, dim3(a.Bq, kHeads / 2), dim3(256), 0, stream, a);
 }

@@ -258,3 +258,28 @@ def test_topk_rows_over_two_ctas():
     for i in range(len(rows)):
         check_topk_exact(lo[i], scores[i], vis[i], 2048)
     assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
+
+
+@pytest.mark.parametrize("kv", ["fp8", "bf16"])
+def test_mla_two_splits_merged_by_a_cta_pair(kv):
+    """64 queries with top_k = 512 take two KV splits, merged inside the decode kernel by
+    the cluster of the two split CTAs. Rows shorter than half of top_k leave the second
+    split with no valid key (weight zero); a row of one token too."""
+    import deepseek_sparse_attention_head_b200 as dsa
+    lens = tuple([1, 100, 255, 256, 257, 700] + [300 + 37 * i for i in range(58)])
+    sp = CaseSpec(f"pair_{kv}", lens, top_k=512, kv_dtype=kv, idx_dtype=kv, seed=44,
+                  out_dtype="fp32" if kv == "bf16" else "bf16")
+    case = generate(sp)
+    assert dsa.mla_num_splits(case["Bq"], 512) == 2
+    vis = oracle.visible_lengths(case)
+    rng = np.random.default_rng(45)
+    logical = np.full((case["Bq"], 512), -1, dtype=np.int64)
+    for q in range(case["Bq"]):
+        n = min(512, int(vis[q]))
+        logical[q, :n] = rng.choice(int(vis[q]), size=n, replace=False)
+    phys = oracle.pagemap(case, logical)
+    from tests.gpu_path import GpuCase
+    out, lse, err = GpuCase(case).mla(phys)
+    assert err == 0
+    ref_out, ref_lse = oracle.mla_sparse_attention(case, phys)
+    check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"])

@@ -33,14 +33,17 @@ def _selection(case, seed):
     return oracle.pagemap(case, logical).astype(np.int32)
 
 
-@pytest.mark.parametrize("nq", [3, 160])       # several KV splits per query / one split each
-def test_stalled_wait_times_out_and_the_next_call_is_correct(nq):
+# several KV splits per query merged by the combine kernel / two splits merged inside the
+# kernel by a CTA pair / one split each
+@pytest.mark.parametrize("nq,splits", [(3, "many"), (64, "pair"), (160, "one")])
+def test_stalled_wait_times_out_and_the_next_call_is_correct(nq, splits):
     import deepseek_sparse_attention_head_b200 as dsa
     case = generate(CaseSpec(f"timeout_{nq}", (700,) * nq, top_k=512, n_planted=0, seed=71))
     t = to_torch(case, "cuda")
     phys = torch.from_numpy(_selection(case, 3)).cuda()
     Bq = case["Bq"]
-    assert (dsa.mla_num_splits(Bq, case["top_k"]) > 1) == (nq == 3)
+    n = dsa.mla_num_splits(Bq, case["top_k"])
+    assert {"many": n > 2, "pair": n == 2, "one": n == 1}[splits]
     ws = dsa.alloc_workspace(dsa.mla_workspace_size(Bq, case["top_k"]))
     out = torch.full((Bq, H, DV), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((Bq, H), float("nan"), dtype=torch.float32, device="cuda")
