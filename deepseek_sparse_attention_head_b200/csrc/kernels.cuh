@@ -39,7 +39,7 @@ struct TopkArgs {
   // long-row gather (chunks > 1): per-query candidate count, largest key - threshold,
   // threshold, and candidate buffers [Bq, cand_cap]; counts and maxima start at zero
   int chunks;
-  int pair;   // 1: each row over a cluster of two CTAs (chunks == 1 only)
+  int pair;   // > 1: each row over a cluster of that many CTAs (chunks == 1 only)
   int cand_cap;
   uint32_t* g_cnt;
   uint32_t* g_rmax;
@@ -163,7 +163,8 @@ cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMa
                            int grid, cudaStream_t stream, int* launches);
 // Chunks per row of the long-row top-k (1 = one CTA per query) and its candidate capacity.
 int topk_chunks(int Bq, int64_t L_max, int sms);
-// 1 when each row's gather is split over a cluster of two CTAs (all pairs in one wave).
+// CTAs per row's cluster (2, 4 or 8) when each row's gather is split over a cluster (all
+// clusters in one wave), else 0.
 int topk_pairs(int Bq, int64_t L_max, int sms);
 int topk_candidate_capacity();
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches);

@@ -539,20 +539,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pagemap_kernel(const TopkAr
   select_whole_row(sm, a, rw);
 }
 
-// Rows gathered by a cluster of two CTAs (query = cluster index): both derive the same
-// threshold, each gathers half of the row straight into the first CTA's candidate buffer
-// (distributed shared memory, its counters and atomics), and after the cluster barrier the
-// first CTA selects and emits. One SM pulls a row at ~16 B/cycle, so two halve the gather.
-// Every branch taken before the barriers depends only on the row, the same in both CTAs.
+// Rows gathered by a cluster of C = 2, 4 or 8 CTAs (query = cluster index): all derive the
+// same threshold, each gathers one C-th of the row straight into the first CTA's candidate
+// buffer (distributed shared memory, its counters and atomics), and after the cluster
+// barrier the first CTA selects and emits. One SM pulls a row at ~16 B/cycle, so C of them
+// divide the gather by C. Every branch taken before the barriers depends only on the row,
+// the same in every CTA of the cluster.
 __global__ void __launch_bounds__(kTopkThreads) topk_pair_kernel(const TopkArgs a) {
   extern __shared__ uint8_t topk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const unsigned rank = cluster.block_rank();
+  const int C = static_cast<int>(cluster.num_blocks());
   pdl_trigger();
   pdl_wait();   // scores come from the indexer
-  const TopkRow rw = topk_row(a, static_cast<int>(blockIdx.x >> 1));
+  const TopkRow rw = topk_row(a, static_cast<int>(blockIdx.x) / C);
   if (rw.vis <= rw.K) {
     if (rank == 0) topk_dense(a, rw);
     return;
@@ -561,9 +563,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pair_kernel(const TopkArgs 
     if (rank == 0) select_whole_row(sm, a, rw);
     return;
   }
-  const int mid = min(rw.vis, ((rw.vis >> 1) + 15) & ~15);   // a multiple of 4: 16-byte loads stay aligned
-  const int lo = rank == 0 ? 0 : mid;
-  const int hi = rank == 0 ? mid : rw.vis;
+  const int part = ((rw.vis + C - 1) / C + 15) & ~15;   // a multiple of 4: 16-byte loads stay aligned
+  const int lo = min(rw.vis, static_cast<int>(rank) * part);
+  const int hi = min(rw.vis, lo + part);
   float4 first[kGatherU / 4];
   gather_load(rw.row, lo, hi, first);   // in flight while the threshold is derived
   const uint32_t thr = row_threshold_small(sm, rw.row, rw.vis, rw.K);
@@ -574,7 +576,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_pair_kernel(const TopkArgs 
   cluster.sync();   // the first CTA's counters are zero before either half adds to them
   TopkSmem& dst = rank == 0 ? sm : *cluster.map_shared_rank(&sm, 0);
   gather_range(rw.row, lo, hi, thr, &dst.n_cand, dst.cand_key, dst.cand_idx, kCand, &dst.rmax, first);
-  cluster.sync();   // both halves' candidates are in the first CTA's buffer
+  cluster.sync();   // every part's candidates are in the first CTA's buffer
   if (rank != 0) return;
   const uint32_t n_c = sm.n_cand;
   if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand)) {
@@ -670,19 +672,24 @@ int topk_chunks(int Bq, int64_t L_max, int sms) {
 }
 
 int topk_pairs(int Bq, int64_t L_max, int sms) {
-  // every pair resident at once (one 1024-thread CTA per SM), rows long enough to split
-  return Bq > 0 && sms > 0 && 2LL * Bq <= sms && L_max >= 32768 ? 1 : 0;
+  // every cluster resident at once (one 1024-thread CTA per SM), at least 16K keys per
+  // CTA for pairs and 8K for larger clusters
+  if (Bq <= 0 || sms <= 0) return 0;
+  for (int c = 8; c >= 4; c >>= 1)
+    if (static_cast<int64_t>(c) * Bq <= sms && L_max >= 8192LL * c) return c;
+  return 2LL * Bq <= sms && L_max >= 32768 ? 2 : 0;
 }
 
 int topk_candidate_capacity() { return kCand; }
 
 cudaError_t launch_topk(const TopkArgs& a, int Bq, cudaStream_t stream, int* launches) {
   const int smem = static_cast<int>(sizeof(TopkSmem));
-  if (a.chunks <= 1 && a.pair) {
+  if (a.chunks <= 1 && a.pair > 1) {
     cudaError_t e = set_smem_once<topk_pair_kernel>(smem);
     if (e != cudaSuccess) return e;
     ++*launches;
-    return launch_pdl_cluster(topk_pair_kernel, dim3(2 * Bq), dim3(kTopkThreads), smem, stream, 2u, a);
+    return launch_pdl_cluster(topk_pair_kernel, dim3(a.pair * Bq), dim3(kTopkThreads), smem, stream,
+                              static_cast<unsigned>(a.pair), a);
   }
   if (a.chunks <= 1) {
     cudaError_t e = set_smem_once<topk_pagemap_kernel>(smem);

@@ -241,21 +241,25 @@ def test_topk_many_queries_mixed_rows():
     assert np.array_equal(ph.astype(np.int64), oracle.pagemap(case, lo.astype(np.int64)))
 
 
-def test_topk_rows_over_two_ctas():
-    """Rows of 40K keys for a few queries take the layout where a cluster of two CTAs
-    gathers each row's halves into one candidate buffer: a constant row (the buffer
-    overflows and the first CTA falls back to the whole-row select after the cluster
-    barrier), few distinct values (ties at the k-th), a near-constant row, all-negative
-    scores, a random row with an odd visible length, and a row shorter than top_k."""
+# rows x keys per row -> CTAs per row's cluster: 40 x 40K -> 2, 6 x 40K -> 4, 3 x 70K -> 8
+@pytest.mark.parametrize("n_rows,L,cluster", [(40, 40000, 2), (6, 40000, 4), (3, 70000, 8)])
+def test_topk_rows_over_a_cta_cluster(n_rows, L, cluster):
+    """Long rows for up to a wave of CTA clusters: each row's gather is split over a cluster
+    of 2, 4 or 8 CTAs writing into one candidate buffer. Rows cycle through a constant row
+    (the buffer overflows and the first CTA falls back to the whole-row select after the
+    cluster barrier), few distinct values (ties at the k-th), a near-constant row,
+    all-negative scores, a random row with an odd visible length and a row shorter than
+    top_k."""
     rng = np.random.default_rng(7)
-    L = 40000
-    rows = [np.full(L, 0.5), rng.choice([0.25, 0.5, 1.0], size=L), rng.standard_normal(L) * 1e-3 + 7.0,
-            -np.abs(rng.standard_normal(L)), rng.standard_normal(L), rng.standard_normal(L)]
-    scores = np.stack(rows).astype(np.float32)
-    vis = np.array([L, L - 5, 39000, L, 33333, 1500])
+    kinds = [lambda: np.full(L, 0.5), lambda: rng.choice([0.25, 0.5, 1.0], size=L),
+             lambda: rng.standard_normal(L) * 1e-3 + 7.0, lambda: -np.abs(rng.standard_normal(L)),
+             lambda: rng.standard_normal(L), lambda: rng.standard_normal(L)]
+    vis_of = [L, L - 5, L - 1000, L, L - 6667, 1500]
+    scores = np.stack([kinds[i % 6]() for i in range(n_rows)]).astype(np.float32)
+    vis = np.array([vis_of[i % 6] for i in range(n_rows)])
     case, lo, ph, err = _topk_on_scores(scores, vis, 2048)
     assert err == 0
-    for i in range(len(rows)):
+    for i in range(n_rows):
         check_topk_exact(lo[i], scores[i], vis[i], 2048)
     assert np.array_equal(ph, oracle.pagemap(case, lo.astype(np.int64)))
 
