@@ -174,10 +174,13 @@ dsa_status run_indexer(const dsa_paging* pg, const void* q_idx, dsa_dtype dt, co
       !make_map(&tq, q_idx, cdt, es, kDimIdx, static_cast<uint64_t>(Bq) * kHeads, box_cols, kHeads))
     return DSA_ERR_CUDA;
   unsigned int* err = err_word(ws);
-  int32_t* prefix = reinterpret_cast<int32_t*>(ws + lay.prefix);
-  cudaError_t e = launch_plan(pg->seq_lens, pg->q_pos, pg->B, pg->n_q, pg->max_pages_per_seq,
-                              indexer_tile_tokens(fp8, pg->n_q), prefix, err, st, &g_launches);
-  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  int32_t* prefix = nullptr;   // up to indexer_prefix_rows() rows the indexer builds it itself
+  if (pg->B > indexer_prefix_rows()) {
+    prefix = reinterpret_cast<int32_t*>(ws + lay.prefix);
+    cudaError_t e = launch_plan(pg->seq_lens, pg->q_pos, pg->B, pg->n_q, pg->max_pages_per_seq,
+                                indexer_tile_tokens(fp8, pg->n_q), prefix, err, st, &g_launches);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+  }
   IndexerArgs a;
   a.B = pg->B;
   a.n_q = pg->n_q;

@@ -29,6 +29,7 @@ namespace dsa {
 constexpr int kEpiWarps = 8;                 // two groups of four, alternating accumulators
 constexpr int kIdxThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kIdxTmemCols = 512;       // accumulators of 64 * min(n_q, 4) columns each
+constexpr int kPrefixRows = 1023;            // rows whose work-item prefix a CTA builds itself
 
 // KC: 128-byte K-chunks per row (1 = fp8, 2 = bf16). QG: queries per group (1 for decode,
 // 4 for chunked prefill). Decode needs only one query per group, so its query slots and
@@ -60,7 +61,9 @@ struct IdxCfg {
   static constexpr int kMaxAcc = 8;
   static constexpr int kNumBars = 2 * kStages + 2 * kBSlots + 2 * kMaxAcc + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
+  // the work-item prefix when the kernel builds it itself (up to kPrefixRows rows)
+  static constexpr int kOffPrefix = kOffMisc + 64;
+  static constexpr int kSmem = kOffPrefix + 4 * (kPrefixRows + 1) + 1024;  // + slack to align the base to 1024
 };
 static_assert(IdxCfg<1, 1>::kHalves / IdxCfg<1, 1>::kUnitHalves == 1 &&
                   IdxCfg<1, 4>::kHalves / IdxCfg<1, 4>::kUnitHalves == 2 &&
@@ -95,8 +98,8 @@ struct TileWalker {
   int max_pages, tile_tok, n_q;
   int b, gt, end, base, bound, len, tiles;
   int vis_b, vis_g, gvis;   // the group whose visible length gvis is cached
-  __device__ void init(const IndexerArgs& a, int tile_tokens, int begin, int stop) {
-    prefix = a.tile_prefix;
+  __device__ void init(const IndexerArgs& a, const int32_t* item_prefix, int tile_tokens, int begin, int stop) {
+    prefix = item_prefix;
     seq_lens = a.seq_lens;
     q_pos = a.q_pos;
     n_q = a.n_q;
@@ -213,14 +216,59 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   pdl_trigger();
   pdl_wait();   // the tile prefix comes from the plan kernel
 
-  const int total = a.tile_prefix[a.B];
+  // the work-item prefix: from the plan kernel, or built here for up to kPrefixRows rows
+  // (each CTA scans the rows' item counts itself; CTA 0 also checks the inputs)
+  const int32_t* prefix = a.tile_prefix;
+  if (prefix == nullptr) {
+    int32_t* sp = reinterpret_cast<int32_t*>(smem + C::kOffPrefix);
+    int* wsum = reinterpret_cast<int*>(smem + C::kOffMisc + 16);   // 10 warp totals
+    const int groups = QG == 1 ? 1 : (a.n_q + QG - 1) / QG;
+    const int tid = threadIdx.x;
+    int carry = 0;
+    for (int base = 0; base < a.B; base += kIdxThreads) {
+      const int b = base + tid;
+      int v = 0;
+      if (b < a.B) v = groups * ((row_len(a.seq_lens, b, a.max_pages) + kTileTok - 1) / kTileTok);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+      }
+      if (lane == 31) wsum[warp] = v;
+      __syncthreads();
+      int before = carry, tot = 0;
+      for (int w = 0; w < kIdxThreads / 32; ++w) {
+        if (w < warp) before += wsum[w];
+        tot += wsum[w];
+      }
+      if (b < a.B) sp[b + 1] = before + v;
+      carry += tot;
+      __syncthreads();
+    }
+    if (tid == 0) sp[0] = 0;
+    if (blockIdx.x == 0) {
+      for (int b = tid; b < a.B; b += kIdxThreads) {
+        const int raw = a.seq_lens[b];
+        if (raw < 0 || raw > a.max_pages * kPage) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(raw));
+      }
+      if (a.q_pos != nullptr)
+        for (int q = tid; q < a.B * a.n_q; q += kIdxThreads) {
+          const int L = row_len(a.seq_lens, q / a.n_q, a.max_pages);
+          const int p = a.q_pos[q];
+          if (p < 0 || p >= L) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(p));
+        }
+    }
+    __syncthreads();
+    prefix = sp;
+  }
+  const int total = prefix[a.B];
   const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
   const int t_begin = min(total, static_cast<int>(blockIdx.x) * per);
   const int t_end = min(total, t_begin + per);
 
   if (t_begin < t_end) {
     TileWalker<QG> walk;
-    walk.init(a, kTileTok, t_begin, t_end);
+    walk.init(a, prefix, kTileTok, t_begin, t_end);
 
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer (whole warp)
@@ -408,7 +456,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       for (int j = 0; j < QG; ++j) qvis[j] = 0;
       bool ok = true;
       TileWalker<QG, false> w2, w4;
-      w2.init(a, kTileTok, t_begin, t_end);
+      w2.init(a, prefix, kTileTok, t_begin, t_end);
       // pages of this thread's tokens in every half of the next tile of walker w (-1 past the end)
       auto tile_pages = [&](TileWalker<QG, false>& w, int (&p)[H]) {
         int bb, gg, tt, LL;
@@ -594,6 +642,8 @@ int indexer_tile_tokens(bool fp8, int n_q) {
   if (n_q == 1) return fp8 ? IdxCfg<1, 1>::kTileTok : IdxCfg<2, 1>::kTileTok;
   return fp8 ? IdxCfg<1, 4>::kTileTok : IdxCfg<2, 4>::kTileTok;
 }
+
+int indexer_prefix_rows() { return kPrefixRows; }
 
 int indexer_query_groups(int n_q) { return n_q == 1 ? 1 : (n_q + 3) / 4; }
 

@@ -19,7 +19,8 @@ struct IndexerArgs {
   const float* k_scale;
   float* scores;
   int64_t L_max;
-  const int32_t* tile_prefix;  // [B+1] exclusive prefix of query groups x ceil(len / tile tokens)
+  const int32_t* tile_prefix;  // [B+1] exclusive prefix of query groups x ceil(len / tile tokens),
+                               // or null: the kernel builds it (B <= indexer_prefix_rows())
   unsigned int* err;
 };
 
@@ -157,6 +158,8 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
 // kernels it queued to *launches.
 // Tokens per indexer tile for this cache type and query count (the plan's tile unit).
 int indexer_tile_tokens(bool fp8, int n_q);
+// Rows up to which the indexer builds its work-item prefix itself (no plan kernel).
+int indexer_prefix_rows();
 cudaError_t launch_plan(const int32_t* seq_lens, const int32_t* q_pos, int B, int n_q, int max_pages, int tile_tok,
                         int32_t* tile_prefix, unsigned int* err, cudaStream_t stream, int* launches);
 cudaError_t launch_indexer(bool fp8, const CUtensorMap& tmap_k, const CUtensorMap& tmap_q, const IndexerArgs& a,

@@ -35,6 +35,9 @@ SMALL = {
     # token, in the longer rows whole runs of tiles, and are skipped by every role
     "prefill_spread": CaseSpec("prefill_spread", (5000, 3000, 1200), top_k=256, n_q=9,
                                q_pos=(0, 100, 255, 256, 511, 700, 900, 1100, 1199), n_planted=0, seed=41),
+    # more rows than an indexer CTA builds its work-item prefix for: the plan kernel builds it
+    "many_rows_plan": CaseSpec("many_rows_plan", tuple((i * 37) % 97 + 1 for i in range(1100)), top_k=32,
+                               seed=46),
     "prefill_spread_bf16": CaseSpec("prefill_spread_bf16", (700, 2100), top_k=128, n_q=5,
                                     q_pos=(3, 255, 256, 511, 699),
                                     idx_dtype="bf16", kv_dtype="bf16", out_dtype="fp32", n_planted=0, seed=42),
@@ -287,3 +290,22 @@ def test_mla_two_splits_merged_by_a_cta_pair(kv):
     assert err == 0
     ref_out, ref_lse = oracle.mla_sparse_attention(case, phys)
     check_attention(out, lse, ref_out, ref_lse, case["kv_dtype"])
+
+
+@pytest.mark.parametrize("rows", [3, 1100])      # prefix built by the indexer / by the plan kernel
+def test_indexer_reports_lengths_and_positions_out_of_range(rows):
+    """A sequence length past the block table and a causal position past its row's length
+    are reported as DSA_ERR_DEVICE_BOUNDS (and clamped), for a prefix built by each indexer
+    CTA and for one built by the plan kernel."""
+    import deepseek_sparse_attention_head_b200 as dsa
+    from tests.gpu_path import GpuCase
+    case = generate(CaseSpec(f"bad_len_{rows}", tuple(40 + i % 50 for i in range(rows)), top_k=16, n_q=2,
+                             q_pos=(3, 30), n_planted=0, seed=47))
+    g = GpuCase(case)
+    assert g.indexer()[1] == 0
+    g.t["seq_lens"][1] = case["max_pages"] * 64 + 5
+    assert g.indexer()[1] == dsa.DSA_ERR_DEVICE_BOUNDS
+    g.t["seq_lens"][1] = int(case["seq_lens"][1])
+    assert g.indexer()[1] == 0
+    g.t["q_pos"][2 * rows - 1] = 10_000
+    assert g.indexer()[1] == dsa.DSA_ERR_DEVICE_BOUNDS
