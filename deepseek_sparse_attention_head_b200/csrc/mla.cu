@@ -7,7 +7,8 @@
 //
 // Design (sm_100a): grid = (query, split); a CTA walks 64-row tiles of its share of the
 // index list through two tile buffers, with warp-specialised roles:
-//   warps 5-12 loaders, all on every tile, tiles alternating between the two buffers.
+//   warps 5.. loaders (8, or 12 for the fp8 cache with a scale plane), all on every tile,
+//   tiles alternating between the two buffers.
 //             Each thread keeps 9 sixteen-byte pieces of each of the next two tiles in
 //             flight (plain global loads issued two tiles ahead), then turns fp8 codes into
 //             fp16 (exact) x a per-row multiplier s_g / 2^E_j and stores them 128-byte
@@ -36,12 +37,13 @@
 namespace dsa {
 
 constexpr int kMlaTile = 64;
-constexpr int kMlaWarps = 13;
-constexpr int kMlaThreads = kMlaWarps * 32;
 constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp0 = 5;                 // loaders: warps 5 .. 12
-constexpr int kLoadThreads = 256;
-constexpr int kBatchPieces = 9;               // 16-byte pieces per loader thread and batch
+constexpr int kLoadWarp0 = 5;                 // loaders: warps 5 .. 4 + NL (NL = 8 or 12 loader warps)
+// Threads of the decode kernel with NL loader warps: 4 softmax warps, the tcgen05 warp, the loaders.
+__host__ __device__ constexpr int mla_threads(int nl) { return (kLoadWarp0 + nl) * 32; }
+// Loader warps per cache layout: a warp keeps only so many loads in flight, so more loader
+// warps pull a tile's rows faster; the 656-byte packed rows divide over 8 only.
+__host__ __device__ constexpr int mla_loaders(int kvf) { return kvf == kKvFp8 ? 12 : 8; }
 constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,128); O^T: cols [128, 384)
 constexpr uint32_t kTmemO = 128;
 constexpr int kNoExp = -100000;               // "no valid row seen yet"
@@ -66,7 +68,7 @@ constexpr int kMlaSmem = kOffIdxList + kIdxListCap * 4 + 1024;
 static_assert(kOffKV % 1024 == 0 && kKVBytes % 1024 == 0, "alignment");
 static_assert(kIdxListCap % kMlaTile == 0, "list capacity");
 static_assert(kMlaSmem <= 232448, "shared memory");
-static_assert(kLoadThreads * kBatchPieces == kMlaTile * 36, "an fp8 tile is one batch");
+
 
 __device__ __forceinline__ uint32_t swz(int row, int unit) {  // 128-byte swizzle inside an 8-row atom
   return static_cast<uint32_t>(row * 128 + ((unit ^ (row & 7)) << 4));
@@ -126,10 +128,14 @@ __device__ __forceinline__ void dequant4_f16(uint32_t w, __half2 m2, uint32_t& o
 // KVF: the latent cache layout, kKvBf16, kKvFp8 (576 E4M3 codes per row + a [rows, 5] fp32
 // scale plane) or kKvFp8Packed (656-byte rows: 512 codes, four fp32 scales, 64 bf16 rope).
 template <int KVF>
-__global__ void __launch_bounds__(kMlaThreads, 1)
+__global__ void __maxnreg__(mla_loaders(KVF) == 12 ? 96 : 128)   // 17 warps: 96 registers fit each sub-partition
     mla_decode_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaArgs a) {
   constexpr bool FP8 = KVF != kKvBf16;            // fp16 operands from E4M3 codes
   constexpr bool PACKED = KVF == kKvFp8Packed;
+  constexpr int NL = mla_loaders(KVF);
+  constexpr int kMlaThreads = mla_threads(NL);
+  constexpr int kLoadThreads = NL * 32;
+  constexpr int kPerQuad = 1 + NL / 4;            // epilogue warps per TMEM lane quadrant
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_ready, 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 8);
+      mbar_init(&kv_full[i], NL);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 4);
       mbar_init(&p_full[i], 4);
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     const uint32_t lb = static_cast<uint32_t>(quad * 32) << 16;
     tc_fence_after();
 #pragma unroll 1
-    for (int k = r; k < 8; k += 3) {
+    for (int k = r; k < 8; k += kPerQuad) {
       const int d = k >> 1, half = k & 1;
       const int dim = d * 128 + quad * 32 + lane;
       float v[32];
@@ -568,7 +574,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     constexpr int kRowPieces = PACKED ? 40 : (FP8 ? 36 : 72);
     constexpr int kRowBytes = PACKED ? kPackedRowBytes : (FP8 ? kDimK : 2 * kDimK);
     constexpr int kBatches = FP8 ? 1 : 2;
-    constexpr int kPieces = PACKED ? 10 : kBatchPieces;   // per thread and batch
+    constexpr int kPieces = kMlaTile * kRowPieces / (kLoadThreads * kBatches);   // per thread and batch
     static_assert(kLoadThreads * kPieces * kBatches == kMlaTile * kRowPieces, "a tile is whole batches");
     uint4 rawA[kPieces], rawB[kPieces];
     float scA[kKvGroups], scB[kKvGroups];
@@ -723,7 +729,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     }
     __syncwarp();
     // the output epilogue with the softmax warps (they publish the per-head scales first)
-    if (bar_and(kEpiBar, kEpiThreads, good) != 0 && !a.pair) write_out(warp <= kLoadWarp0 + 3 ? 1 : 2);
+    if (bar_and(kEpiBar, kEpiThreads, good) != 0 && !a.pair) write_out(1 + (warp - kLoadWarp0) / 4);
   }
 
   if (ntiles == 0 && a.pair) {
@@ -792,14 +798,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     // a split with nothing selected sends nothing (its weight is 0) but writes its own heads
     const bool epi = (warp < 4 || warp >= kLoadWarp0) && sPair[kPairGood] != 0.0f;
     const bool send = epi && ntiles > 0;
-    const int part = warp < 4 ? 0 : (warp <= kLoadWarp0 + 3 ? 1 : 2);   // three warps per lane quadrant
+    const int part = warp < 4 ? 0 : 1 + (warp - kLoadWarp0) / 4;   // kPerQuad warps per lane quadrant
     const int quad = warp & 3;
     const uint32_t lb = static_cast<uint32_t>(quad * 32) << 16;
     float* recv = reinterpret_cast<float*>(sKV);                        // [32 heads][512 dims]
     if (send) {
       float* precv = cluster.map_shared_rank(recv, static_cast<unsigned>(peer));
 #pragma unroll 1
-      for (int d = part; d < 4; d += 3) {
+      for (int d = part; d < 4; d += kPerQuad) {
         const int dim = d * 128 + quad * 32 + lane;
         float v[32];
         tmem_ld32(tmem + kTmemO + lb + d * 64 + peer * 32, v);
@@ -815,7 +821,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     tc_fence_after();
     if (epi) {
 #pragma unroll 1
-      for (int d = part; d < 4; d += 3) {
+      for (int d = part; d < 4; d += kPerQuad) {
         const int dim = d * 128 + quad * 32 + lane;
         float v[32];
         tmem_ld32(tmem + kTmemO + lb + d * 64 + split * 32, v);
@@ -905,12 +911,13 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
 
 template <int KVF>
 static cudaError_t launch_mla_t(const CUtensorMap& tq, const MlaArgs& a, cudaStream_t stream) {
+  constexpr int threads = mla_threads(mla_loaders(KVF));
   cudaError_t e = set_smem_once<mla_decode_kernel<KVF>>(kMlaSmem);
   if (e != cudaSuccess) return e;
   if (a.pair)
-    return launch_pdl_cluster(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, 2u,
+    return launch_pdl_cluster(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(threads), kMlaSmem, stream, 2u,
                               tq, a);
-  return launch_pdl(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(kMlaThreads), kMlaSmem, stream, tq, a);
+  return launch_pdl(mla_decode_kernel<KVF>, dim3(a.Bq * a.nsplit), dim3(threads), kMlaSmem, stream, tq, a);
 }
 
 cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cudaStream_t stream, int* launches) {
