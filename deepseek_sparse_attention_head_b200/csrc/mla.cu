@@ -43,7 +43,7 @@ constexpr int kLoadWarp0 = 5;                 // loaders: warps 5 .. 4 + NL (NL 
 __host__ __device__ constexpr int mla_threads(int nl) { return (kLoadWarp0 + nl) * 32; }
 // Loader warps per cache layout: a warp keeps only so many loads in flight, so more loader
 // warps pull a tile's rows faster; the 656-byte packed rows divide over 8 only.
-__host__ __device__ constexpr int mla_loaders(int kvf) { return kvf == kKvFp8 ? 12 : 8; }
+__host__ __device__ constexpr int mla_loaders(int kvf) { return kvf != kKvFp8Packed ? 12 : 8; }
 constexpr uint32_t kMlaTmemCols = 512;        // S[2]: cols [0,128); O^T: cols [128, 384)
 constexpr uint32_t kTmemO = 128;
 constexpr int kNoExp = -100000;               // "no valid row seen yet"
