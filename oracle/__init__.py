@@ -6,5 +6,6 @@ from .dsa_oracle import (  # noqa: F401
     visible_lengths, physical_slots, pagemap, indexer_scores, topk_logical,
     mla_sparse_attention, mla_partials, combine_partials, mla_sparse_attention_split,
     decode_layer, encode_e4m3, quantize_e4m3, encode_bf16, rope_interleaved, new_token_positions,
-    physical_slots_rows, rope_quantize_append,
+    physical_slots_rows, rope_quantize_append, shard_candidates, shard_global_select,
+    sharded_decode_layer,
 )

@@ -30,6 +30,11 @@ format, page size or tie rule; these are the plainest readings the rest supports
   * with vis(q) <= top_k every visible token is selected (the dense path);
   * an empty selection gives a zero output and lse = -inf.
 
+The token-sharded step (sharded_decode_layer, the long-context extension): each row's
+tokens spread over several ranks, a local top-k per rank, an exchange of (score, token)
+candidates, a global selection (ties to the lower global token), each rank's attention
+state over the selected tokens it holds, and the log-sum-exp merge of those states.
+
 The step before the path (rope_quantize_append, the next step after the hot path): the new
 tokens' projected indexer queries and keys and latent rows get partial interleaved RoPE
 ("Show HN: colibri", features: MLA with partial interleaved RoPE) on their 64 rope columns
@@ -416,3 +421,77 @@ def rope_quantize_append(case: dict, new: dict, base: float = 10000.0) -> dict:
         qm[..., DV:] = rope_interleaved(qm[..., DV:], pos[:, None], base)
         out["q_mla"] = encode_bf16(qm)
     return out
+
+
+# ----------------------------------------------------------------------------------
+# token-sharded decode: one long sequence spread over several ranks, one exchange step
+#
+# The pages say only that the context reaches 1M tokens (Russian news item on colibri);
+# how such a context is spread over GPUs is not on them. The plainest reading that keeps
+# the step's result unchanged: each rank holds a contiguous range of every row's tokens,
+# scores and ranks only its own tokens, and the ranks exchange their best candidates and
+# then their attention states.
+
+def shard_candidates(scores_row: np.ndarray, lo: int, hi: int, top_k: int):
+    """One rank's local selection of one query row: the min(top_k, hi - lo) best of its
+    tokens [lo, hi) (topk_logical on the slice), as (score, global token) pairs padded
+    with (-inf, -1) to top_k entries."""
+    local = topk_logical(scores_row[None, lo:hi], np.array([hi - lo]), top_k)[0]
+    ok = local >= 0
+    tok = np.where(ok, local + lo, -1)
+    sc = np.where(ok, scores_row[np.maximum(tok, 0)], -np.inf)
+    return sc, tok
+
+
+def shard_global_select(cand_score: np.ndarray, cand_token: np.ndarray, top_k: int) -> np.ndarray:
+    """Global selection from every rank's candidates (flattened): the min(top_k, #valid)
+    best, descending score, ties to the lower global token; tokens -1 are padding."""
+    ok = cand_token >= 0
+    sc, tok = cand_score[ok], cand_token[ok]
+    order = np.lexsort((tok, -sc))
+    out = np.full(top_k, -1, dtype=np.int64)
+    k = min(top_k, tok.size)
+    out[:k] = tok[order[:k]]
+    return out
+
+
+def sharded_decode_layer(case: dict, bounds: np.ndarray, queries=None):
+    """The decode step with every row's tokens spread over R ranks.
+
+    bounds: int [B, R + 1], nondecreasing from 0 to seq_lens[b]; rank r holds tokens
+    [bounds[b, r], bounds[b, r + 1]) of row b. Every query sees its whole row (no q_pos).
+    Steps: (1) each rank scores its tokens (a token's score does not depend on where it
+    is stored, so the scores are the whole row's, sliced); (2) each rank's local top-k
+    as (score, global token) candidates; (3) the exchange: all ranks see all candidates;
+    (4) the global selection among them; (5) each rank's attention state over the
+    selected tokens it holds (mla_partials); (6) the log-sum-exp merge of the R states
+    (combine_partials).
+    Returns dict(logical [n, top_k] global tokens in descending-score order, physical,
+    owner [n, top_k] rank of each selected token (-1 unused), out, lse)."""
+    if case.get("q_pos") is not None:
+        raise ValueError("the token-sharded step takes no causal positions")
+    queries = np.arange(case["Bq"]) if queries is None else np.asarray(queries)
+    bounds = np.asarray(bounds, dtype=np.int64)
+    R = bounds.shape[1] - 1
+    K = case["top_k"]
+    scores = indexer_scores(case, queries)
+    n = len(queries)
+    logical = np.full((n, K), -1, dtype=np.int64)
+    owner = np.full((n, K), -1, dtype=np.int64)
+    out = np.zeros((n, H, DV))
+    lse = np.full((n, H), -np.inf)
+    for i, q in enumerate(queries):
+        b = q // case["n_q"]
+        cands = [shard_candidates(scores[i], bounds[b, r], bounds[b, r + 1], K) for r in range(R)]
+        sel = shard_global_select(np.concatenate([c[0] for c in cands]), np.concatenate([c[1] for c in cands]), K)
+        logical[i] = sel
+        ok = sel >= 0
+        owner[i][ok] = np.searchsorted(bounds[b], sel[ok], side="right") - 1
+        states = []
+        for r in range(R):
+            mine = sel[ok & (owner[i] == r)]
+            states.append(mla_partials(case, physical_slots(case["block_table"][b], mine), q))
+        out[i], lse[i] = combine_partials([s[0] for s in states], [s[1] for s in states], [s[2] for s in states])
+    physical = np.stack([physical_slots(case["block_table"][q // case["n_q"]], logical[i])
+                         for i, q in enumerate(queries)])
+    return dict(scores=scores, logical=logical, physical=physical, owner=owner, out=out, lse=lse)

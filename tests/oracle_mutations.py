@@ -252,3 +252,42 @@ _ORIG_ROPE = od.rope_interleaved
 MUTATIONS["rope_rotates_halves_not_pairs"] = lambda: _set("rope_interleaved", _rope_half_split)
 MUTATIONS["rope_turns_the_other_way"] = lambda: _set("rope_interleaved", _rope_reversed)
 MUTATIONS["append_slot_one_page_off"] = lambda: _set("physical_slots_rows", _slots_one_page_off)
+
+
+def _shard_select_ties_high(cand_score, cand_token, top_k):
+    ok = cand_token >= 0
+    sc, tok = cand_score[ok], cand_token[ok]
+    order = np.lexsort((-tok, -sc))
+    out = np.full(top_k, -1, dtype=np.int64)
+    k = min(top_k, tok.size)
+    out[:k] = tok[order[:k]]
+    return out
+
+
+def _shard_candidates_local_tokens(scores_row, lo, hi, top_k):
+    local = od.topk_logical(scores_row[None, lo:hi], np.array([hi - lo]), top_k)[0]
+    ok = local >= 0
+    tok = np.where(ok, local, -1)
+    sc = np.where(ok, scores_row[np.maximum(local + lo, 0)], -np.inf)
+    return sc, tok
+
+
+def _shard_candidates_one_short(scores_row, lo, hi, top_k):
+    sc, tok = _shard_candidates_copy(scores_row, lo, hi, top_k)
+    if hi - lo >= top_k:
+        sc[-1], tok[-1] = -np.inf, -1
+    return sc, tok
+
+
+def _shard_candidates_copy(scores_row, lo, hi, top_k):
+    local = od.topk_logical(scores_row[None, lo:hi], np.array([hi - lo]), top_k)[0]
+    ok = local >= 0
+    tok = np.where(ok, local + lo, -1)
+    sc = np.where(ok, scores_row[np.maximum(tok, 0)], -np.inf)
+    return sc, tok
+
+
+MUTATIONS["shard_select_ties_to_higher_token"] = lambda: _set("shard_global_select", _shard_select_ties_high)
+MUTATIONS["shard_candidates_keep_local_tokens"] = lambda: _set("shard_candidates", _shard_candidates_local_tokens)
+MUTATIONS["shard_candidates_one_short"] = lambda: _set("shard_candidates", _shard_candidates_one_short)
+CONTROLS["control_shard_candidates_copy"] = lambda: _set("shard_candidates", _shard_candidates_copy)

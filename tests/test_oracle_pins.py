@@ -427,6 +427,68 @@ def test_poison_never_reaches_outputs():
     assert np.all(np.abs(r["out"]) < 10)
 
 
+# ---------------------------------------------------------------- token-sharded step
+
+def test_shard_candidates_by_hand():
+    row = np.array([5.0, 1.0, 7.0, 7.0, 2.0, 9.0, 3.0])
+    sc, tok = oracle.shard_candidates(row, 2, 6, 3)          # slice [7, 7, 2, 9] of tokens 2..5
+    assert list(tok) == [5, 2, 3] and list(sc) == [9.0, 7.0, 7.0]
+    sc, tok = oracle.shard_candidates(row, 5, 7, 4)          # two tokens: padded
+    assert list(tok) == [5, 6, -1, -1] and list(sc[:2]) == [9.0, 3.0] and np.all(np.isneginf(sc[2:]))
+    sc, tok = oracle.shard_candidates(row, 3, 3, 2)          # an empty shard
+    assert list(tok) == [-1, -1]
+
+
+def test_shard_global_select_by_hand():
+    sc = np.array([4.0, 6.0, -np.inf, 6.0, 1.0, 6.0])
+    tok = np.array([10, 31, -1, 7, 2, 40])
+    assert list(oracle.shard_global_select(sc, tok, 3)) == [7, 31, 40]
+    assert list(oracle.shard_global_select(sc, tok, 2)) == [7, 31]
+    assert list(oracle.shard_global_select(sc, tok, 7)) == [7, 31, 40, 10, 2, -1, -1]
+
+
+_SHARD_LAYOUTS = {
+    "one_rank": [[0, 300], [0, 130]],
+    "equal_pages": [[0, 128, 256, 300], [0, 64, 128, 130]],
+    "empty_ranks": [[0, 0, 192, 300], [0, 130, 130, 130]],
+    "shards_shorter_than_top_k": [[0, 64, 128, 192, 256, 300], [0, 64, 64, 128, 128, 130]],
+}
+
+
+@pytest.mark.parametrize("layout", sorted(_SHARD_LAYOUTS))
+def test_sharded_step_equals_unsharded(layout):
+    """The union of the ranks' local top-k holds a global top-k, and the log-sum-exp merge
+    of per-rank softmax states is the softmax over their union: the sharded step gives the
+    unsharded step's selection exactly and its attention to rounding."""
+    case = generate(CaseSpec("t", (300, 130), top_k=64, seed=31, kv_dtype="fp8"))
+    bounds = np.array(_SHARD_LAYOUTS[layout])
+    a = oracle.decode_layer(case)
+    b = oracle.sharded_decode_layer(case, bounds)
+    assert np.array_equal(a["logical"], b["logical"])
+    assert np.array_equal(a["physical"], b["physical"])
+    assert np.allclose(a["out"], b["out"], rtol=1e-12, atol=1e-14)
+    assert np.allclose(a["lse"], b["lse"], rtol=1e-12)
+    for i in range(case["Bq"]):
+        sel, own = b["logical"][i], b["owner"][i]
+        ok = sel >= 0
+        assert np.all(bounds[i][own[ok]] <= sel[ok]) and np.all(sel[ok] < bounds[i][own[ok] + 1])
+
+
+def test_sharded_step_dense_rows_take_every_token():
+    case = generate(CaseSpec("t", (100, 40), top_k=128, seed=32))
+    r = oracle.sharded_decode_layer(case, np.array([[0, 64, 100], [0, 0, 40]]))
+    assert sorted(r["logical"][0][r["logical"][0] >= 0]) == list(range(100))
+    assert sorted(r["logical"][1][r["logical"][1] >= 0]) == list(range(40))
+
+
+def test_sharded_step_ties_go_to_the_lower_global_token():
+    """All scores equal (zero caches): whatever the layout, tokens 0..k-1 are selected."""
+    case = blank_case([320], top_k=8)
+    for bounds in ([0, 128, 320], [0, 256, 320], [0, 64, 128, 192, 256, 320]):
+        r = oracle.sharded_decode_layer(case, np.array([bounds]))
+        assert list(r["logical"][0]) == list(range(8))
+
+
 # ---------------------------------------------------------------- the step before the path
 
 def test_e4m3_encoder_round_trips_ties_to_even_and_saturates():
