@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa_b20
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_WORKSPACE, \
     DSA_ERR_DEVICE_BOUNDS, DSA_ERR_TIMEOUT = range(7)
 DSA_BF16, DSA_FP8_E4M3, DSA_FP32, DSA_FP8_E4M3_ROPE_BF16 = range(4)
-DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_PAGEMAP, DSA_OP_LAYER = range(4)
+DSA_OP_INDEXER, DSA_OP_TOPK, DSA_OP_PAGEMAP, DSA_OP_LAYER, DSA_OP_SHARD_LOCAL, DSA_OP_SHARD_SELECT = range(6)
 
 PAGE_SIZE = 64
 HEADS = 64
@@ -65,6 +65,9 @@ _SIGNATURES = {
                                 _vp, _vp, _vp, _vp, _sz, _vp]),
     "dsa_rope_quantize_append": (_i32, [_PP, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                                         _vp]),
+    "dsa_shard_local_topk": (_i32, [_PP, _vp, _i64, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "dsa_shard_select": (_i32, [_PP, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "dsa_shard_merge": (_i32, [_i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp]),
     "dsa_workspace_size": (_sz, [_PP, _i64, _i32, _i32]),
     "mla_workspace_size": (_sz, [_i32, _i32]),
     "mla_num_splits": (_i32, [_i32, _i32]),
@@ -282,3 +285,37 @@ def dsa_decode_layer(paging: Paging, q_idx, q_scale, head_w, k_cache, k_scale, q
                                workspace.numel(), _stream(stream))
     _check(st, "dsa_decode_layer")
     return out
+
+
+# ---------------------------------------------------------------------- token-sharded decode
+
+def dsa_shard_local_topk(paging: Paging, scores: torch.Tensor, top_k: int, token_offset: torch.Tensor,
+                         cand_score: torch.Tensor, cand_token: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """This rank's top-k as exchange candidates: (score, global token) pairs [Bq, top_k]."""
+    st = _lib.dsa_shard_local_topk(paging.ref(), _ptr(scores), int(scores.shape[-1]), int(top_k),
+                                   _ptr(token_offset), _ptr(cand_score), _ptr(cand_token), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "dsa_shard_local_topk")
+    return cand_score, cand_token
+
+
+def dsa_shard_select(paging: Paging, n_ranks: int, rank: int, all_score: torch.Tensor, all_token: torch.Tensor,
+                     top_k: int, token_offset: torch.Tensor, physical_out: torch.Tensor, workspace: torch.Tensor,
+                     logical_out=None, stream=None):
+    """Global selection among every rank's candidates [n_ranks, Bq, top_k]; this rank's
+    winners as slots of its own caches (first, then -1)."""
+    st = _lib.dsa_shard_select(paging.ref(), int(n_ranks), int(rank), _ptr(all_score), _ptr(all_token), int(top_k),
+                               _ptr(token_offset), _ptr(physical_out), _ptr(logical_out), _ptr(workspace),
+                               workspace.numel(), _stream(stream))
+    _check(st, "dsa_shard_select")
+    return physical_out
+
+
+def dsa_shard_merge(all_out: torch.Tensor, all_lse: torch.Tensor, out: torch.Tensor, lse=None, stream=None):
+    """Log-sum-exp merge of every rank's (out fp32 [Bq, 64, 512], lse [Bq, 64]) state."""
+    n_ranks, Bq = int(all_out.shape[0]), int(all_out.shape[1])
+    st = _lib.dsa_shard_merge(Bq, n_ranks, _ptr(all_out), _ptr(all_lse), _ptr(out), _dtype_code(out), _ptr(lse),
+                              _stream(stream))
+    _check(st, "dsa_shard_merge")
+    return out
+

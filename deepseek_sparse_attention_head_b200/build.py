@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdsa_b200.so")
-SOURCES = ["api.cu", "indexer.cu", "topk.cu", "mla.cu", "append.cu"]
+SOURCES = ["api.cu", "indexer.cu", "topk.cu", "mla.cu", "append.cu", "shard.cu"]
 HEADERS = ["common.cuh", "kernels.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -132,7 +132,11 @@ Layout layout_for(int B, int64_t Bq, int64_t L_max, int top_k, int op, int nspli
     l.physical = off;
     off += up256(static_cast<size_t>(Bq) * top_k * 4);
   }
-  if (op == DSA_OP_TOPK || op == DSA_OP_LAYER) {
+  if (op == DSA_OP_SHARD_LOCAL) {
+    l.logical = off;
+    off += up256(static_cast<size_t>(Bq) * top_k * 4);
+  }
+  if (op == DSA_OP_TOPK || op == DSA_OP_LAYER || op == DSA_OP_SHARD_LOCAL) {
     const int ch = topk_chunks(static_cast<int>(Bq), L_max, device_sms());
     if (ch > 1) {
       const size_t cap = static_cast<size_t>(topk_candidate_capacity());
@@ -323,9 +327,10 @@ extern "C" {
 
 size_t dsa_workspace_size(const dsa_paging* paging, int64_t L_max, int32_t top_k, int32_t op) {
   if (check_paging(paging) != DSA_OK) return 0;
-  if (op < DSA_OP_INDEXER || op > DSA_OP_LAYER) return 0;
+  if (op < DSA_OP_INDEXER || op > DSA_OP_SHARD_SELECT) return 0;
   const int64_t Bq = static_cast<int64_t>(paging->B) * paging->n_q;
   int nsplit = 1;
+  if (op == DSA_OP_SHARD_LOCAL && (top_k < 1 || top_k > 16384)) return 0;
   if (op == DSA_OP_LAYER) {
     if (top_k < 1 || top_k > 16384) return 0;
     nsplit = mla_splits_for(static_cast<int>(Bq), top_k, nullptr);
@@ -443,6 +448,91 @@ dsa_status dsa_decode_layer(const dsa_paging* paging, const void* q_idx, dsa_dty
   if (s != DSA_OK) return s;
   return run_mla(static_cast<int>(Bq), q_mla, kv_cache, kv_dtype, kv_scale, num_slots, physical, top_k,
                  softmax_scale, out, out_dtype, lse, ws, lay, nsplit, kps, st);
+}
+
+dsa_status dsa_shard_local_topk(const dsa_paging* local, const float* scores, int64_t L_max, int32_t top_k,
+                                const int32_t* token_offset, float* cand_score, int32_t* cand_token,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  dsa_status s = check_paging(local);
+  if (s != DSA_OK) return s;
+  if (local->q_pos != nullptr) return DSA_ERR_UNSUPPORTED;
+  if (scores == nullptr || L_max < 1 || top_k < 1 || top_k > 16384) return DSA_ERR_INVALID_ARG;
+  if (token_offset == nullptr || cand_score == nullptr || cand_token == nullptr) return DSA_ERR_INVALID_ARG;
+  const int64_t Bq = static_cast<int64_t>(local->B) * local->n_q;
+  const Layout lay = layout_for(local->B, Bq, L_max, top_k, DSA_OP_SHARD_LOCAL, 1);
+  s = check_ws(workspace, ws_bytes, lay.total);
+  if (s != DSA_OK) return s;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* logical = reinterpret_cast<int32_t*>(ws + lay.logical);
+  s = run_topk(local, scores, L_max, top_k, logical, nullptr, ws, lay, false, st);
+  if (s != DSA_OK) return s;
+  ShardCandArgs a;
+  a.Bq = static_cast<int>(Bq);
+  a.n_q = local->n_q;
+  a.top_k = top_k;
+  a.scores = scores;
+  a.L_max = L_max;
+  a.logical = logical;
+  a.token_offset = token_offset;
+  a.cand_score = cand_score;
+  a.cand_token = cand_token;
+  a.err = err_word(ws);
+  return cuda_status(launch_shard_candidates(a, st, &g_launches));
+}
+
+dsa_status dsa_shard_select(const dsa_paging* local, int32_t n_ranks, int32_t rank, const float* all_score,
+                            const int32_t* all_token, int32_t top_k, const int32_t* token_offset,
+                            int32_t* physical_out, int32_t* logical_out, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  g_launches = 0;
+  dsa_status s = check_paging(local);
+  if (s != DSA_OK) return s;
+  if (local->q_pos != nullptr) return DSA_ERR_UNSUPPORTED;
+  if (n_ranks < 1 || rank < 0 || rank >= n_ranks || top_k < 1 || top_k > 16384) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(n_ranks) * top_k >= (int64_t(1) << 30)) return DSA_ERR_UNSUPPORTED;
+  if (all_score == nullptr || all_token == nullptr || token_offset == nullptr || physical_out == nullptr)
+    return DSA_ERR_INVALID_ARG;
+  s = check_ws(workspace, ws_bytes, layout_for(local->B, 0, 0, top_k, DSA_OP_SHARD_SELECT, 1).total);
+  if (s != DSA_OK) return s;
+  ShardSelectArgs a;
+  a.Bq = local->B * local->n_q;
+  a.n_q = local->n_q;
+  a.top_k = top_k;
+  a.n_ranks = n_ranks;
+  a.rank = rank;
+  a.all_score = all_score;
+  a.all_token = all_token;
+  a.token_offset = token_offset;
+  a.seq_lens = local->seq_lens;
+  a.block_table = local->block_table;
+  a.max_pages = local->max_pages_per_seq;
+  a.num_pages = local->num_pages;
+  a.physical = physical_out;
+  a.logical = logical_out;
+  a.err = err_word(workspace);
+  a.in_smem = shard_select_smem_bytes(n_ranks * top_k) > 0 ? 1 : 0;
+  return cuda_status(launch_shard_select(a, static_cast<cudaStream_t>(stream), &g_launches));
+}
+
+dsa_status dsa_shard_merge(int32_t Bq, int32_t n_ranks, const float* all_out, const float* all_lse, void* out,
+                           dsa_dtype out_dtype, float* lse, void* stream) {
+  g_launches = 0;
+  if (Bq < 1 || n_ranks < 1 || all_out == nullptr || all_lse == nullptr || out == nullptr) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(Bq) * kHeads >= (int64_t(1) << 31) / n_ranks) return DSA_ERR_UNSUPPORTED;
+  if (out_dtype != DSA_BF16 && out_dtype != DSA_FP32) return DSA_ERR_INVALID_ARG;
+  if (!aligned(all_out, 16) || !aligned(out, out_dtype == DSA_FP32 ? 16 : 8) || !aligned(all_lse, 4))
+    return DSA_ERR_INVALID_ARG;
+  ShardMergeArgs a;
+  a.Bq = Bq;
+  a.n_ranks = n_ranks;
+  a.all_out = all_out;
+  a.all_lse = all_lse;
+  a.out = out;
+  a.out_fp32 = out_dtype == DSA_FP32 ? 1 : 0;
+  a.lse = lse;
+  return cuda_status(launch_shard_merge(a, static_cast<cudaStream_t>(stream), &g_launches));
 }
 
 dsa_status dsa_get_error(void* workspace, void* stream) {

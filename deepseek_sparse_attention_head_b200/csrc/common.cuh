@@ -435,6 +435,29 @@ __device__ __forceinline__ int query_vis(const int32_t* q_pos, int q, int L) {
   return v < 0 ? 0 : (v > L ? L : v);
 }
 
+// Larger float -> larger unsigned key (negative values bit-flipped, positives get the top bit).
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Reserves `n` consecutive slots of a shared counter for each lane of a converged, full
+// warp with one atomic per warp; returns the lane's first slot.
+__device__ __forceinline__ uint32_t warp_reserve(uint32_t* counter, uint32_t n) {
+  const int lane = static_cast<int>(threadIdx.x & 31);
+  uint32_t incl = n;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+  uint32_t base = 0;
+  if (lane == 31 && total != 0u) base = atomicAdd(counter, total);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  return base + incl - n;
+}
+
 // Physical page of logical page p of row b; out-of-range entries are recorded and
 // replaced by page 0 so no access leaves the cache.
 __device__ __forceinline__ int checked_page(const int32_t* block_table, int b, int p, int max_pages,

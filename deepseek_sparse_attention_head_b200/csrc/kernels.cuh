@@ -182,4 +182,44 @@ cudaError_t launch_mla(int kvf, const CUtensorMap& tmap_q, const MlaArgs& a, cud
 cudaError_t launch_rope_quantize_append(const AppendArgs& a, int Bq, cudaStream_t stream, int* launches);
 int mla_tile_keys();  // index-list entries per MLA tile (splits are whole tiles)
 
+// Token-sharded decode (shard.cu).
+struct ShardCandArgs {
+  int Bq, n_q, top_k;
+  const float* scores;           // [Bq, L_max] this rank's indexer scores
+  int64_t L_max;
+  const int32_t* logical;        // [Bq, top_k] this rank's local selection (-1 unused)
+  const int32_t* token_offset;   // [B] global token of each row's local token 0
+  float* cand_score;             // [Bq, top_k] out: score, -inf where unused
+  int32_t* cand_token;           // [Bq, top_k] out: global token, -1 where unused
+  unsigned int* err;
+};
+struct ShardSelectArgs {
+  int Bq, n_q, top_k, n_ranks, rank;
+  const float* all_score;        // [n_ranks, Bq, top_k] every rank's candidates
+  const int32_t* all_token;
+  const int32_t* token_offset;   // [B] this rank's offsets
+  const int32_t* seq_lens;       // [B] this rank's local lengths
+  const int32_t* block_table;    // [B, max_pages] this rank's block table
+  int max_pages, num_pages;
+  int32_t* physical;             // [Bq, top_k] out: this rank's winners' slots, then -1
+  int32_t* logical;              // [Bq, top_k] out (or null): the global selection
+  unsigned int* err;
+  int in_smem;                   // the candidates of a row are staged in shared memory
+};
+struct ShardMergeArgs {
+  int Bq, n_ranks;
+  const float* all_out;          // [n_ranks, Bq, 64, 512] every rank's normalised output
+  const float* all_lse;          // [n_ranks, Bq, 64]
+  void* out;                     // [Bq, 64, 512] bf16 or fp32
+  int out_fp32;
+  float* lse;                    // [Bq, 64] or null
+};
+constexpr int kShardSelectSmemCap = 227 * 1024;
+// Dynamic shared memory of the select kernel with a row's n_cand candidates staged, or 0
+// when they do not fit (the kernel then reads them from global memory on every pass).
+int shard_select_smem_bytes(int n_cand);
+cudaError_t launch_shard_candidates(const ShardCandArgs& a, cudaStream_t stream, int* launches);
+cudaError_t launch_shard_select(const ShardSelectArgs& a, cudaStream_t stream, int* launches);
+cudaError_t launch_shard_merge(const ShardMergeArgs& a, cudaStream_t stream, int* launches);
+
 }  // namespace dsa

@@ -1,0 +1,312 @@
+// Token-sharded decode of long sequences: each row's tokens are spread over R ranks (one
+// GPU each), and one exchange step joins them (the long-context extension of the decode
+// step; the pages say only that the context reaches 1M tokens, Russian news item on
+// colibri). Per rank:
+//   1. indexer scores and a local top-k over the rank's own tokens (the usual stages);
+//   2. shard_candidates_kernel: the local winners as (score, global token) pairs, the
+//      payload of the exchange;
+//   3. (all ranks gather every rank's payload: a collective outside this library)
+//   4. shard_select_kernel: the global top-k among all candidates, ties to the lower
+//      global token, identical on every rank; the winners this rank holds are mapped to
+//      its physical slots (first in the list, -1 after);
+//   5. MLA sparse decode over those slots (fp32 output + lse: the rank's softmax state);
+//   6. (all ranks gather every rank's state)
+//   7. shard_merge_kernel: the log-sum-exp merge of the R states.
+// The union of the local top-k lists holds a global top-k, and merging softmax states by
+// their log-sum-exp gives the softmax over the union, so the result is the unsharded step's.
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+
+namespace dsa {
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelBins = 256;   // 8-bit radix digits, four passes per 32-bit key
+
+// ------------------------------------------------------------------ candidates
+
+__global__ void shard_candidates_kernel(const ShardCandArgs a) {
+  pdl_trigger();
+  pdl_wait();   // the local selection comes from the top-k kernel
+  const int64_t total = static_cast<int64_t>(a.Bq) * a.top_k;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int q = static_cast<int>(i / a.top_k);
+    const int s = a.logical[i];
+    float sc = -INFINITY;
+    int tok = -1;
+    if (s >= 0 && s < a.L_max) {
+      const int64_t g = static_cast<int64_t>(a.token_offset[q / a.n_q]) + s;
+      if (a.token_offset[q / a.n_q] < 0 || g > 0x7fffffffLL) {
+        record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(a.token_offset[q / a.n_q]));
+      } else {
+        sc = a.scores[static_cast<int64_t>(q) * a.L_max + s];
+        tok = static_cast<int>(g);
+      }
+    }
+    a.cand_score[i] = sc;
+    a.cand_token[i] = tok;
+  }
+}
+
+// ------------------------------------------------------------------ global select
+
+struct SelSmem {
+  uint32_t hist[kSelBins];
+  uint32_t bin, rem, eq, n_valid, n_sel, n_mine, n_eq2;
+};
+
+// Candidate c of query q: entry (r = c / K, i = c % K) of the gathered [R, Bq, K] arrays,
+// read from the shared-memory copy when the row fits there.
+struct CandView {
+  const float* sc;
+  const int32_t* tok;
+  const uint32_t* skey;   // shared copy (or null)
+  const int32_t* stok;
+  int K, Bq, q;
+  __device__ __forceinline__ int64_t gidx(int c) const {
+    const int r = c / K;
+    return (static_cast<int64_t>(r) * Bq + q) * K + (c - r * K);
+  }
+  __device__ __forceinline__ int token(int c) const { return stok ? stok[c] : tok[gidx(c)]; }
+  __device__ __forceinline__ uint32_t key(int c) const { return skey ? skey[c] : order_key(sc[gidx(c)]); }
+};
+
+// The k-th largest (1-based, k >= 1) of the keys key(c) over the candidates with take(c),
+// exact, by four 8-bit radix passes. Returns the key; *need = how many candidates equal
+// to it belong to the top k, *n_equal = how many there are. Whole CTA.
+template <typename Key, typename Take>
+__device__ uint32_t radix_kth(SelSmem& sm, int n, uint32_t k, Key key, Take take, uint32_t* need,
+                              uint32_t* n_equal) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  uint32_t prefix = 0u, pmask = 0u, remaining = k, eq = 0u;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < kSelBins; i += kSelThreads) sm.hist[i] = 0u;
+    __syncthreads();
+    for (int c = tid; c < n; c += kSelThreads) {
+      if (!take(c)) continue;
+      const uint32_t u = key(c);
+      if ((u & pmask) == prefix) atomicAdd(&sm.hist[(u >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l holds bins [8 (31 - l), 8 (31 - l) + 8): lane 0 the largest digits
+      const int base = 8 * (31 - lane);
+      uint32_t h[8], s = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        h[j] = sm.hist[base + j];
+        s += h[j];
+      }
+      uint32_t incl = s;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      const uint32_t above = incl - s;   // keys in larger digits than this lane's
+      if (above < remaining && remaining <= incl) {
+        uint32_t acc = above;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+          if (acc + h[j] >= remaining) {
+            sm.bin = static_cast<uint32_t>(base + j);
+            sm.rem = remaining - acc;
+            sm.eq = h[j];
+            break;
+          }
+          acc += h[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= sm.bin << shift;
+    pmask |= 0xFFu << shift;
+    remaining = sm.rem;
+    eq = sm.eq;
+    __syncthreads();   // sm.bin / sm.rem are rewritten by the next pass
+  }
+  *need = remaining;
+  *n_equal = eq;
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSelectArgs a) {
+  extern __shared__ uint8_t sel_smem_raw[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(sel_smem_raw);
+  const int tid = threadIdx.x;
+  const int q = blockIdx.x;
+  const int b = q / a.n_q;
+  const int K = a.top_k;
+  const int n = a.n_ranks * K;
+  pdl_trigger();
+  pdl_wait();   // the gathered candidates may come from an earlier kernel on the stream
+
+  CandView v{a.all_score, a.all_token, nullptr, nullptr, K, a.Bq, q};
+  if (a.in_smem) {
+    uint32_t* skey = reinterpret_cast<uint32_t*>(sel_smem_raw + sizeof(SelSmem));
+    int32_t* stok = reinterpret_cast<int32_t*>(skey + n);
+    for (int c = tid; c < n; c += kSelThreads) {
+      const int64_t g = v.gidx(c);
+      skey[c] = order_key(a.all_score[g]);
+      stok[c] = a.all_token[g];
+    }
+    v.skey = skey;
+    v.stok = stok;
+  }
+  if (tid == 0) {
+    sm.n_valid = 0u;
+    sm.n_sel = 0u;
+    sm.n_mine = 0u;
+    sm.n_eq2 = 0u;
+  }
+  __syncthreads();
+  {
+    uint32_t cnt = 0u;
+    for (int c = tid; c < n; c += kSelThreads) cnt += v.token(c) >= 0 ? 1u : 0u;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if ((tid & 31) == 0 && cnt != 0u) atomicAdd(&sm.n_valid, cnt);
+  }
+  __syncthreads();
+  const uint32_t n_valid = sm.n_valid;
+  const uint32_t k = n_valid < static_cast<uint32_t>(K) ? n_valid : static_cast<uint32_t>(K);
+
+  // selection rule: all valid candidates (k == n_valid), else score key above kth, or equal
+  // to it and among the `need` lowest global tokens of those equal
+  bool all = k == n_valid;
+  uint32_t kth = 0u, need = 0u, n_equal = 0u, kth2 = 0u, need2 = 0u, n_equal2 = 0u;
+  bool all_equal = true;
+  auto valid = [&](int c) { return v.token(c) >= 0; };
+  if (!all) {
+    kth = radix_kth(sm, n, k, [&](int c) { return v.key(c); }, valid, &need, &n_equal);
+    all_equal = need == n_equal;
+    if (!all_equal) {
+      // ties at the k-th score: the `need` lowest tokens (larger key = lower token)
+      kth2 = radix_kth(
+          sm, n, need, [&](int c) { return ~static_cast<uint32_t>(v.token(c)); },
+          [&](int c) { return valid(c) && v.key(c) == kth; }, &need2, &n_equal2);
+    }
+  }
+
+  const int off = a.token_offset[b];
+  int len = a.seq_lens[b];
+  len = len < 0 ? 0 : (len > a.max_pages * kPage ? a.max_pages * kPage : len);
+  int32_t* lo_row = a.logical ? a.logical + static_cast<int64_t>(q) * K : nullptr;
+  int32_t* ph_row = a.physical + static_cast<int64_t>(q) * K;
+  for (int c = tid; c < n; c += kSelThreads) {
+    const int tok = v.token(c);
+    bool pick = tok >= 0;
+    if (pick && !all) {
+      const uint32_t u = v.key(c);
+      if (u < kth) {
+        pick = false;
+      } else if (u == kth && !all_equal) {
+        const uint32_t u2 = ~static_cast<uint32_t>(tok);
+        // distinct tokens make kth2 unique; duplicates (an invalid layout) are capped
+        pick = u2 > kth2 || (u2 == kth2 && atomicAdd(&sm.n_eq2, 1u) < need2);
+      }
+    }
+    if (!pick) continue;
+    const uint32_t p = atomicAdd(&sm.n_sel, 1u);
+    if (p >= k) continue;
+    if (lo_row) lo_row[p] = tok;
+    if (c / K != a.rank) continue;
+    const int s = tok - off;
+    if (s < 0 || s >= len) {
+      record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(tok));
+      continue;
+    }
+    const int slot = checked_page(a.block_table, b, s >> 6, a.max_pages, a.num_pages, a.err) * kPage + (s & 63);
+    ph_row[atomicAdd(&sm.n_mine, 1u)] = slot;
+  }
+  __syncthreads();
+  const int n_sel = static_cast<int>(sm.n_sel < k ? sm.n_sel : k);
+  const int n_mine = static_cast<int>(sm.n_mine);
+  if (lo_row)
+    for (int i = n_sel + tid; i < K; i += kSelThreads) lo_row[i] = -1;
+  for (int i = n_mine + tid; i < K; i += kSelThreads) ph_row[i] = -1;
+}
+
+// ------------------------------------------------------------------ merge
+
+// 128 threads per (query, head), four columns each; R states merged per thread.
+constexpr int kMergeHeadsPerCta = 2;
+
+__global__ void __launch_bounds__(128 * kMergeHeadsPerCta) shard_merge_kernel(const ShardMergeArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int hq = blockIdx.x * kMergeHeadsPerCta + static_cast<int>(threadIdx.x >> 7);   // q * 64 + h
+  if (hq >= a.Bq * kHeads) return;
+  const int col = 4 * static_cast<int>(threadIdx.x & 127);
+  const int64_t stride_lse = static_cast<int64_t>(a.Bq) * kHeads;
+  float M = -INFINITY;
+  for (int r = 0; r < a.n_ranks; ++r) M = fmaxf(M, a.all_lse[r * stride_lse + hq]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+  if (M != -INFINITY) {
+    for (int r = 0; r < a.n_ranks; ++r) {
+      const float l = a.all_lse[r * stride_lse + hq];
+      if (l == -INFINITY) continue;
+      const float w = expf(l - M);
+      L += w;
+      const float4 o = *reinterpret_cast<const float4*>(a.all_out + (r * stride_lse + hq) * kDimV + col);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
+    const float inv = 1.f / L;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+  }
+  const int64_t o = static_cast<int64_t>(hq) * kDimV + col;
+  if (a.out_fp32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + o) = acc;
+  } else {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + o) = pk;
+  }
+  if (a.lse && col == 0) a.lse[hq] = M == -INFINITY ? -INFINITY : M + logf(L);
+}
+
+// ------------------------------------------------------------------ launches
+
+int shard_select_smem_bytes(int n_cand) {
+  const int64_t in = static_cast<int64_t>(sizeof(SelSmem)) + static_cast<int64_t>(n_cand) * 8;
+  return in <= kShardSelectSmemCap ? static_cast<int>(in) : 0;
+}
+
+cudaError_t launch_shard_candidates(const ShardCandArgs& a, cudaStream_t stream, int* launches) {
+  const int64_t total = static_cast<int64_t>(a.Bq) * a.top_k;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  ++*launches;
+  return launch_pdl(shard_candidates_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, a);
+}
+
+cudaError_t launch_shard_select(const ShardSelectArgs& a, cudaStream_t stream, int* launches) {
+  const int smem = a.in_smem ? shard_select_smem_bytes(a.n_ranks * a.top_k) : static_cast<int>(sizeof(SelSmem));
+  if (smem > 48 * 1024) {
+    const cudaError_t e = set_smem_once<shard_select_kernel>(kShardSelectSmemCap);
+    if (e != cudaSuccess) return e;
+  }
+  ++*launches;
+  return launch_pdl(shard_select_kernel, dim3(a.Bq), dim3(kSelThreads), smem, stream, a);
+}
+
+cudaError_t launch_shard_merge(const ShardMergeArgs& a, cudaStream_t stream, int* launches) {
+  const int64_t heads = static_cast<int64_t>(a.Bq) * kHeads;
+  ++*launches;
+  return launch_pdl(shard_merge_kernel, dim3(static_cast<unsigned>((heads + kMergeHeadsPerCta - 1) / kMergeHeadsPerCta)),
+                    dim3(128 * kMergeHeadsPerCta), 0, stream, a);
+}
+
+}  // namespace dsa

@@ -24,12 +24,6 @@
 
 namespace dsa {
 
-// Larger float -> larger unsigned key (negative values bit-flipped, positives get the top bit).
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 constexpr int kTopkThreads = 1024;
 constexpr int kHistBins = 4096;
 constexpr int kCand = 12288;  // candidates kept in shared memory
@@ -116,23 +110,6 @@ __device__ __forceinline__ void select_bin(TopkSmem& sm, uint32_t remaining) {
     above += cs[i];
   }
   __syncthreads();
-}
-
-// Reserves `n` consecutive slots of a shared counter for each lane of a converged, full
-// warp with one atomic per warp; returns the lane's first slot.
-__device__ __forceinline__ uint32_t warp_reserve(uint32_t* counter, uint32_t n) {
-  const int lane = static_cast<int>(threadIdx.x & 31);
-  uint32_t incl = n;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += t;
-  }
-  const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-  uint32_t base = 0;
-  if (lane == 31 && total != 0u) base = atomicAdd(counter, total);
-  base = __shfl_sync(0xffffffffu, base, 31);
-  return base + incl - n;
 }
 
 // Per-row context shared by the phases below.

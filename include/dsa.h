@@ -69,7 +69,9 @@ typedef enum {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_PAGEMAP = 2,
-  DSA_OP_LAYER = 3
+  DSA_OP_LAYER = 3,
+  DSA_OP_SHARD_LOCAL = 4,    /* dsa_shard_local_topk  */
+  DSA_OP_SHARD_SELECT = 5    /* dsa_shard_select      */
 } dsa_op;
 
 /*
@@ -207,6 +209,66 @@ dsa_status dsa_decode_layer(const dsa_paging* paging,
                             void* out, dsa_dtype out_dtype, float* lse,
                             int32_t* logical_out, int32_t* physical_out,
                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Token-sharded decode: one long sequence per row spread over R ranks (one GPU each),
+ * joined by one exchange step. The pages say only that the context reaches 1M tokens
+ * (Russian news item on colibri); this split is the library's long-context extension and
+ * its result is the unsharded step's: the union of the ranks' local top-k lists holds a
+ * global top-k, and merging the ranks' softmax states by their log-sum-exp gives the
+ * softmax over the union.
+ *
+ * Rank r holds tokens [token_offset[b], token_offset[b] + seq_lens[b]) of every row b in
+ * its own paged caches, described by its own `local` paging (q_pos must be NULL: every
+ * query sees its whole row). Per decode step, on every rank:
+ *   1. dsa_indexer_scores(local, ...) over the rank's tokens;
+ *   2. dsa_shard_local_topk: local top-k, as (score, global token) candidates;
+ *   3. the caller gathers every rank's candidates (e.g. an NCCL all-gather) into
+ *      all_score / all_token [R, Bq, top_k], rank-major;
+ *   4. dsa_shard_select: the global selection, and this rank's share of it as slots;
+ *   5. mla_sparse_decode over those slots with fp32 `out` and `lse`: the rank's state;
+ *   6. the caller gathers every rank's out [R, Bq, 64, 512] and lse [R, Bq, 64];
+ *   7. dsa_shard_merge: the log-sum-exp merge into the step's output.
+ * Every rank passes identical gathered arrays to steps 4 and 7 and gets identical results.
+ */
+
+/* Step 2: top-k of this rank's scores (as dsa_topk_pagemap) and the exchange payload
+ *  cand_score  device [B*n_q, top_k] fp32: the selected scores, -inf in unused entries
+ *  cand_token  device [B*n_q, top_k] int32: their global tokens token_offset[b] + s, -1 unused
+ *  token_offset device [B] int32 >= 0 (a global token past 2^31 - 1 is a device-side error)
+ * Workspace: dsa_workspace_size(local, L_max, top_k, DSA_OP_SHARD_LOCAL).
+ * DSA_ERR_UNSUPPORTED when local->q_pos is not NULL. */
+dsa_status dsa_shard_local_topk(const dsa_paging* local, const float* scores, int64_t L_max, int32_t top_k,
+                                const int32_t* token_offset, float* cand_score, int32_t* cand_token,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Step 4: the global selection among every rank's candidates
+ *  all_score, all_token  device [n_ranks, B*n_q, top_k] as gathered (rank-major)
+ *  physical_out device [B*n_q, top_k] int32: the physical slots (in `local`'s block table)
+ *               of the selected tokens this rank holds, first, then -1
+ *  logical_out  device [B*n_q, top_k] int32 or NULL: the whole selection as global tokens
+ *               (unordered, -1 after the k selected), the same on every rank
+ * Per query k = min(top_k, valid candidates) are selected: the highest scores, and among
+ * equal scores at the boundary the lower global tokens (unlike dsa_topk_pagemap, whose
+ * boundary ties are arbitrary, so that every rank takes the same decision). A selected
+ * token of this rank outside [token_offset[b], token_offset[b] + seq_lens[b]) is a
+ * device-side error and is dropped. 1 <= n_ranks, 0 <= rank < n_ranks,
+ * n_ranks * top_k < 2^30. Workspace: dsa_workspace_size(local, 0, top_k,
+ * DSA_OP_SHARD_SELECT). DSA_ERR_UNSUPPORTED when local->q_pos is not NULL. */
+dsa_status dsa_shard_select(const dsa_paging* local, int32_t n_ranks, int32_t rank, const float* all_score,
+                            const int32_t* all_token, int32_t top_k, const int32_t* token_offset,
+                            int32_t* physical_out, int32_t* logical_out, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/* Step 7: log-sum-exp merge of the ranks' attention states
+ *  all_out  device [n_ranks, Bq, 64, 512] fp32 (16-byte aligned): each rank's normalised output
+ *  all_lse  device [n_ranks, Bq, 64] fp32: each rank's lse (-inf: no selected token there)
+ *  out      device [Bq, 64, 512] in out_dtype (DSA_BF16, 8-byte aligned, or DSA_FP32,
+ *           16-byte aligned): sum_r exp(lse_r - LSE) out_r, LSE = log sum_r exp(lse_r)
+ *  lse      device [Bq, 64] fp32 LSE, or NULL
+ * A (query, head) with every lse_r = -inf gets out = 0 and lse = -inf. No workspace. */
+dsa_status dsa_shard_merge(int32_t Bq, int32_t n_ranks, const float* all_out, const float* all_lse, void* out,
+                           dsa_dtype out_dtype, float* lse, void* stream);
 
 /* Bytes of workspace `op` needs for this paging (L_max only matters for DSA_OP_INDEXER
  * and DSA_OP_TOPK, where it may be 0). Returns 0 when the arguments are invalid. */

@@ -151,3 +151,61 @@ def test_append_argument_errors():
     assert call(status=ctypes.c_void_p(0x100004)) == dsa.DSA_ERR_INVALID_ARG
     assert _lib.dsa_rope_quantize_append(None, FAKE, FAKE, FAKE, None, 10000.0, FAKE, FAKE, FAKE, FAKE, FAKE,
                                          dsa.DSA_FP8_E4M3, FAKE, None, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_shard_argument_errors():
+    pg = paging(B=2, max_pages=4)
+    ws_l = _lib.dsa_workspace_size(ctypes.byref(pg), 256, 16, dsa.DSA_OP_SHARD_LOCAL)
+    assert ws_l >= 256 + 2 * 16 * 4 and ws_l % 256 == 0
+    assert _lib.dsa_workspace_size(ctypes.byref(pg), 256, 0, dsa.DSA_OP_SHARD_LOCAL) == 0
+    assert _lib.dsa_workspace_size(ctypes.byref(pg), 256, 16, 6) == 0
+    ws_s = _lib.dsa_workspace_size(ctypes.byref(pg), 0, 16, dsa.DSA_OP_SHARD_SELECT)
+    assert ws_s >= 256
+
+    def local(p=pg, top_k=16, offset=FAKE, ws_bytes=ws_l):
+        return _lib.dsa_shard_local_topk(ctypes.byref(p), FAKE, 256, top_k, offset, FAKE, FAKE, FAKE, ws_bytes, None)
+
+    assert local(offset=None) == dsa.DSA_ERR_INVALID_ARG
+    assert local(top_k=0) == dsa.DSA_ERR_INVALID_ARG
+    assert local(top_k=16385) == dsa.DSA_ERR_INVALID_ARG
+    assert local(ws_bytes=ws_l - 1) == dsa.DSA_ERR_WORKSPACE
+    causal = _Paging(2, 1, FAKE, FAKE, FAKE, 4, 64, 8)
+    assert local(p=causal) == dsa.DSA_ERR_UNSUPPORTED
+
+    def select(p=pg, n_ranks=2, rank=0, top_k=16, physical=FAKE, ws_bytes=ws_s):
+        return _lib.dsa_shard_select(ctypes.byref(p), n_ranks, rank, FAKE, FAKE, top_k, FAKE, physical, None, FAKE,
+                                     ws_bytes, None)
+
+    assert select(rank=2) == dsa.DSA_ERR_INVALID_ARG
+    assert select(rank=-1) == dsa.DSA_ERR_INVALID_ARG
+    assert select(n_ranks=0) == dsa.DSA_ERR_INVALID_ARG
+    assert select(physical=None) == dsa.DSA_ERR_INVALID_ARG
+    assert select(n_ranks=1 << 17, top_k=8192) == dsa.DSA_ERR_UNSUPPORTED
+    assert select(ws_bytes=0) == dsa.DSA_ERR_WORKSPACE
+    assert select(p=causal) == dsa.DSA_ERR_UNSUPPORTED
+
+    def merge(Bq=1, n_ranks=2, all_out=FAKE, out=FAKE, dt=dsa.DSA_FP32):
+        return _lib.dsa_shard_merge(Bq, n_ranks, all_out, FAKE, out, dt, None, None)
+
+    assert merge(Bq=0) == dsa.DSA_ERR_INVALID_ARG
+    assert merge(n_ranks=0) == dsa.DSA_ERR_INVALID_ARG
+    assert merge(dt=dsa.DSA_FP8_E4M3) == dsa.DSA_ERR_INVALID_ARG
+    assert merge(all_out=ctypes.c_void_p(0x100004)) == dsa.DSA_ERR_INVALID_ARG
+    assert merge(out=ctypes.c_void_p(0x100008)) == dsa.DSA_ERR_INVALID_ARG        # fp32 out needs 16 bytes
+    assert merge(out=None) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_shard_bounds_are_page_aligned_and_cover_the_row():
+    from deepseek_sparse_attention_head_b200.sharded import shard_bounds
+    assert shard_bounds(1000, 1) == [0, 1000]
+    assert shard_bounds(1000, 2) == [0, 512, 1000]
+    assert shard_bounds(1000, 3) == [0, 384, 768, 1000]
+    assert shard_bounds(100, 4) == [0, 64, 100, 100, 100]
+    assert shard_bounds(0, 3) == [0, 0, 0, 0]
+    for L in (1, 63, 64, 65, 4095, 1 << 20):
+        for R in (1, 2, 3, 8):
+            b = shard_bounds(L, R)
+            assert b[0] == 0 and b[-1] == L and all(x <= y for x, y in zip(b, b[1:]))
+            assert all(x % 64 == 0 or x == L for x in b)   # every shard starts on a page
+    with pytest.raises(ValueError):
+        shard_bounds(10, 0)
