@@ -43,6 +43,9 @@ def parse():
     p.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a CUDA graph")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=200)
+    p.add_argument("--token-shards", type=int, default=0,
+                   help="R > 0: the token-sharded step, every row's tokens over R ranks (under torchrun R must "
+                        "equal the number of ranks; on one GPU the R ranks run in lockstep in this process)")
     return p.parse_args()
 
 
@@ -574,6 +577,193 @@ def run_ours(args, world, rank, local):
     return result
 
 
+def run_token_sharded(args, world, rank, local):
+    """Token-sharded step: every row's tokens spread over R ranks, one exchange step.
+
+    Under torchrun (world == R) each rank runs its share and the exchanges are NCCL
+    all-gathers (eager launches). On one GPU the R ranks run in lockstep in this process,
+    the exchanges become device copies into one gathered buffer, and the whole step is
+    captured in a CUDA graph; each rank's phases are also timed alone, so that the
+    critical path of R GPUs (slowest rank's local phase + slowest rank's select and
+    attention + the merge, exchanges excluded) can be read beside the one-GPU rate.
+    Strong scaling: the total work of a step is fixed."""
+    import deepseek_sparse_attention_head_b200 as dsa
+    from deepseek_sparse_attention_head_b200.sharded import TokenShardedDecode, shard_bounds
+
+    R = args.token_shards
+    if world > 1 and R != world:
+        raise SystemExit("--token-shards must equal the number of ranks under torchrun")
+    case = dsa_inputs.generate(dsa_inputs.spec(args.workload))
+    if case["q_pos"] is not None:
+        raise SystemExit("the token-sharded step takes workloads without causal positions")
+    nbytes = dsa_inputs.algorithmic_bytes(case)
+    t = dsa_inputs.to_torch(case, "cuda")
+    B, Bq, K = case["B"], case["Bq"], case["top_k"]
+    bounds = np.array([shard_bounds(int(L), R) for L in case["seq_lens"]], dtype=np.int64)
+    mine = list(range(R)) if world == 1 else [rank]
+    decs = {}
+    for r in mine:
+        lo, hi = bounds[:, r], bounds[:, r + 1]
+        lens = (hi - lo).astype(np.int32)
+        npg = (lens + 63) // 64
+        lbt = np.full((B, max(1, int(npg.max()))), -1, dtype=np.int32)
+        for b in range(B):
+            lbt[b, :npg[b]] = case["block_table"][b, lo[b] // 64:lo[b] // 64 + npg[b]]
+        paging = dsa.Paging(torch.from_numpy(lens).cuda(), torch.from_numpy(lbt).cuda(), case["num_pages"],
+                            case["n_q"])
+        decs[r] = TokenShardedDecode(paging, torch.from_numpy(lo.astype(np.int32)).cuda(), K, case["softmax_scale"],
+                                     r, R)
+    if world == 1:   # one gathered buffer shared by the emulated ranks
+        for name in ("all_score", "all_token", "all_out", "all_lse"):
+            buf = getattr(decs[0], name)
+            for d in decs.values():
+                setattr(d, name, buf)
+    out_dt = torch.float32 if case["out_dtype"] == "fp32" else torch.bfloat16
+    out = torch.empty(Bq, 64, 512, dtype=out_dt, device="cuda")
+    lse = torch.empty(Bq, 64, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    idx_in = (t["q_idx"], t["q_idx_scale"], t["head_w"], t["k_cache"], t["k_scale"])
+    mla_in = (t["q_mla"], t["kv_cache"], t["kv_scale"])
+
+    def step():
+        if world > 1:
+            decs[rank].step(*idx_in, *mla_in, out, lse)
+            return
+        for d in decs.values():
+            d.local_phase(*idx_in)
+        for r, d in decs.items():
+            d.all_score[r].copy_(d.cand_score)
+            d.all_token[r].copy_(d.cand_token)
+        for d in decs.values():
+            d.select_phase()
+            d.attend_phase(*mla_in)
+        for r, d in decs.items():
+            d.all_out[r].copy_(d.state_out)
+            d.all_lse[r].copy_(d.state_lse)
+        decs[mine[0]].merge_phase(out, lse)   # every rank's merge is the same call
+
+    # warm-up step, eager, counting this process's kernel launches per call
+    launches = 0
+    with torch.cuda.stream(stream):
+        for d in decs.values():
+            dsa.dsa_indexer_scores(d.paging, *idx_in, d.scores, d.ws_index)
+            launches += dsa.dsa_last_launch_count()
+            dsa.dsa_shard_local_topk(d.paging, d.scores, K, d.token_offset, d.cand_score, d.cand_token, d.ws_local)
+            launches += dsa.dsa_last_launch_count()
+        step()
+        for d in decs.values():
+            d.select_phase()
+            launches += dsa.dsa_last_launch_count()
+            d.attend_phase(*mla_in)
+            launches += dsa.dsa_last_launch_count()
+        decs[mine[0]].merge_phase(out, lse)
+        launches += dsa.dsa_last_launch_count()
+    stream.synchronize()
+    for d in decs.values():
+        for w in (d.ws_index, d.ws_local, d.ws_select, d.ws_mla):
+            if dsa.dsa_get_error(w, stream) != 0:
+                raise RuntimeError("device error in the warm-up step")
+
+    graph = None
+    if world == 1 and not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        stream.synchronize()
+
+    def run(n):
+        for _ in range(n):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+
+    with torch.cuda.stream(stream):
+        run(max(3, args.warmup))
+    stream.synchronize()
+    inputs_exceed_l2 = nbytes["total"] > L2_BYTES
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    if inputs_exceed_l2:
+        ms = timed_back_to_back(lambda: run(1), args.steps, stream)
+    else:
+        ms = timed_flushed(lambda: run(1), args.steps, stream, flush)
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_max = max_over_ranks(ms, world)
+
+    per_rank = None
+    if world == 1:
+        # each emulated rank's phases timed alone: 20 calls of the phase captured in one CUDA
+        # graph, replayed a few times on the same stream (device time: a graph per call would
+        # time the host's replay rate for phases of a few microseconds)
+        per_graph, reps = 20, 5
+
+        def graph_ms(fn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(per_graph):
+                    fn()
+            stream.synchronize()
+            with torch.cuda.stream(stream):
+                g.replay()
+            ms_ = timed_back_to_back(g.replay, reps, stream) / (reps * per_graph)
+            del g
+            return ms_
+
+        per_rank = []
+        for d in decs.values():
+            t_idx = graph_ms(lambda: dsa.dsa_indexer_scores(d.paging, *idx_in, d.scores, d.ws_index))
+            t_topk = graph_ms(lambda: dsa.dsa_shard_local_topk(d.paging, d.scores, K, d.token_offset, d.cand_score,
+                                                               d.cand_token, d.ws_local))
+            t_sel = graph_ms(d.select_phase)
+            t_att = graph_ms(lambda: d.attend_phase(*mla_in))
+            per_rank.append({"rank": d.rank, "indexer_ms": t_idx, "local_topk_ms": t_topk, "select_ms": t_sel,
+                             "attend_ms": t_att, "local_ms": t_idx + t_topk, "select_attend_ms": t_sel + t_att})
+        t_merge = graph_ms(lambda: decs[mine[0]].merge_phase(out, lse))
+        crit = (max(p["local_ms"] for p in per_rank) + max(p["select_attend_ms"] for p in per_rank) + t_merge)
+    result = {
+        "metric": METRIC,
+        "value": 1e3 * args.steps / ms_max,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "e4m3 indexer + f16 MLA operands, fp32 accumulate" if case["idx_dtype"] != "bf16" else "bf16",
+        "data": "synthetic (seeded; dsa_inputs)",
+        "config": {
+            "workload": f"{args.workload}: {dsa_inputs.WORKLOAD_NAMES[args.workload]}, token-sharded over {R} ranks",
+            "B": B, "n_q": case["n_q"], "sum_L": int(case["seq_lens"].sum()), "top_k": K,
+            "parallelism": (f"token shards x{R} (NCCL all-gathers)" if world > 1 else
+                            f"token shards x{R} emulated on one GPU (exchanges as device copies)"),
+            "launch": "cuda_graph" if graph is not None else "eager",
+            "l2": "inputs larger than L2" if inputs_exceed_l2 else "L2 flushed before every step",
+            "shard_bounds": bounds.tolist(),
+        },
+        "exchange_bytes_per_rank": {"candidates": Bq * K * 8, "states": Bq * 64 * (512 + 1) * 4},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+        "roofline": None,
+        "e2e": None,
+    }
+    if per_rank is not None:
+        result["per_rank"] = per_rank
+        result["merge_ms"] = t_merge
+        result["critical_path_ms_excluding_exchanges"] = crit
+    if graph is not None:
+        del graph
+    return result
+
+
 # ------------------------------------------------------------------ oracle (CPU baseline / reference arm)
 
 def oracle_threads():
@@ -655,7 +845,7 @@ def main():
         print(json.dumps(run_reference(args, world, rank)), flush=True)
         return 0
     world, rank, local = dist_setup(args)
-    res = run_ours(args, world, rank, local)
+    res = run_token_sharded(args, world, rank, local) if args.token_shards > 0 else run_ours(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

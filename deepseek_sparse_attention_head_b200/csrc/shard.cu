@@ -16,6 +16,8 @@
 // their log-sum-exp gives the softmax over the union, so the result is the unsharded step's.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace dsa {
@@ -53,43 +55,149 @@ __global__ void shard_candidates_kernel(const ShardCandArgs a) {
 
 struct SelSmem {
   uint32_t hist[kSelBins];
-  uint32_t bin, rem, eq, n_valid, n_sel, n_mine, n_eq2;
+  uint32_t bin, rem, eq, n_valid, n_sel, n_mine, n_eq2, kmin, kmax;
 };
 
-// Candidate c of query q: entry (r = c / K, i = c % K) of the gathered [R, Bq, K] arrays,
-// read from the shared-memory copy when the row fits there.
-struct CandView {
+// Candidates of query q: candidate c is entry (r = c / K, i = c % K) of the gathered
+// [R, Bq, K] arrays. Two sources give every thread the same number of visits (so that
+// warp-wide ballots stay converged), each visit f(c, key, token) with token -1 past the end:
+//  * RegCands<P>: rows of at most P x 1024 candidates live in registers, P per thread
+//    (c = tid + 1024 j), loaded once with all loads in flight;
+//  * MemCands: longer rows, read from a shared-memory copy when it fits, else from global
+//    memory on every visit.
+__device__ __forceinline__ int64_t cand_gidx(int c, int K, int Bq, int q) {
+  const int r = c / K;
+  return (static_cast<int64_t>(r) * Bq + q) * K + (c - r * K);
+}
+
+template <int P>
+struct RegCands {
+  uint32_t key[P];
+  int32_t tok[P];
+  __device__ __forceinline__ void load(const ShardSelectArgs& a, int n, int q) {
+#pragma unroll
+    for (int j = 0; j < P; ++j) {
+      const int c = static_cast<int>(threadIdx.x) + j * kSelThreads;
+      float sc = 0.f;
+      tok[j] = -1;
+      if (c < n) {
+        const int64_t g = cand_gidx(c, a.top_k, a.Bq, q);
+        sc = __ldg(a.all_score + g);
+        tok[j] = __ldg(a.all_token + g);
+      }
+      key[j] = order_key(sc);
+    }
+  }
+  template <typename F>
+  __device__ __forceinline__ void visit(F f) const {
+#pragma unroll
+    for (int j = 0; j < P; ++j) f(static_cast<int>(threadIdx.x) + j * kSelThreads, key[j], tok[j]);
+  }
+};
+
+struct MemCands {
   const float* sc;
-  const int32_t* tok;
+  const int32_t* tk;
   const uint32_t* skey;   // shared copy (or null)
   const int32_t* stok;
-  int K, Bq, q;
-  __device__ __forceinline__ int64_t gidx(int c) const {
-    const int r = c / K;
-    return (static_cast<int64_t>(r) * Bq + q) * K + (c - r * K);
+  int n, K, Bq, q;
+  __device__ void load(const ShardSelectArgs& a, uint8_t* smem_tail) {
+    if (!a.in_smem) return;
+    uint32_t* k_ = reinterpret_cast<uint32_t*>(smem_tail);
+    int32_t* t_ = reinterpret_cast<int32_t*>(k_ + n);
+    constexpr int kU = 8;   // eight candidates per thread in flight at once
+    for (int c0 = threadIdx.x; c0 < n; c0 += kU * kSelThreads) {
+      float s_[kU];
+      int32_t tt[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * kSelThreads;
+        if (c < n) {
+          const int64_t g = cand_gidx(c, K, Bq, q);
+          s_[u] = __ldg(sc + g);
+          tt[u] = __ldg(tk + g);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + u * kSelThreads;
+        if (c < n) {
+          k_[c] = order_key(s_[u]);
+          t_[c] = tt[u];
+        }
+      }
+    }
+    skey = k_;
+    stok = t_;
   }
-  __device__ __forceinline__ int token(int c) const { return stok ? stok[c] : tok[gidx(c)]; }
-  __device__ __forceinline__ uint32_t key(int c) const { return skey ? skey[c] : order_key(sc[gidx(c)]); }
+  template <typename F>
+  __device__ void visit(F f) const {
+    for (int c0 = 0; c0 < n; c0 += kSelThreads) {
+      const int c = c0 + static_cast<int>(threadIdx.x);
+      uint32_t u = 0u;
+      int32_t t = -1;
+      if (c < n) {
+        if (skey) {
+          u = skey[c];
+          t = stok[c];
+        } else {
+          const int64_t g = cand_gidx(c, K, Bq, q);
+          u = order_key(sc[g]);
+          t = tk[g];
+        }
+      }
+      f(c, u, t);
+    }
+  }
 };
 
-// The k-th largest (1-based, k >= 1) of the keys key(c) over the candidates with take(c),
-// exact, by four 8-bit radix passes. Returns the key; *need = how many candidates equal
-// to it belong to the top k, *n_equal = how many there are. Whole CTA.
-template <typename Key, typename Take>
-__device__ uint32_t radix_kth(SelSmem& sm, int n, uint32_t k, Key key, Take take, uint32_t* need,
+// The k-th largest (1-based, k >= 1) of key(u, t) over the candidates with take(u, t),
+// exact. The radix runs over r = key - (smallest taken key), from the highest bit in which
+// the taken keys differ, in 8-bit digits (candidates gathered from every rank's top-k have
+// close scores, so their keys share most leading bits). Returns the key; *need = how many
+// candidates equal to it belong to the top k, *n_equal = how many there are. Whole CTA.
+template <typename Src, typename Key, typename Take>
+__device__ uint32_t radix_kth(SelSmem& sm, const Src& src, uint32_t k, Key key, Take take, uint32_t* need,
                               uint32_t* n_equal) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  if (tid == 0) {
+    sm.kmin = 0xFFFFFFFFu;
+    sm.kmax = 0u;
+  }
+  __syncthreads();
+  {
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    src.visit([&](int, uint32_t u, int32_t t) {
+      if (take(u, t)) {
+        const uint32_t v = key(u, t);
+        lo = v < lo ? v : lo;
+        hi = v > hi ? v : hi;
+      }
+    });
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) {
+      atomicMin(&sm.kmin, lo);
+      atomicMax(&sm.kmax, hi);
+    }
+  }
+  __syncthreads();
+  const uint32_t kmin = sm.kmin;
+  const uint32_t span = sm.kmax - kmin;
+  int top = span == 0u ? 0 : 32 - __clz(span);   // every r fits in bits [0, top)
   uint32_t prefix = 0u, pmask = 0u, remaining = k, eq = 0u;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (true) {
+    const int lo_bit = top > 8 ? top - 8 : 0;
+    const uint32_t dm = (1u << (top - lo_bit)) - 1u;   // top - lo_bit in [0, 8]
     for (int i = tid; i < kSelBins; i += kSelThreads) sm.hist[i] = 0u;
     __syncthreads();
-    for (int c = tid; c < n; c += kSelThreads) {
-      if (!take(c)) continue;
-      const uint32_t u = key(c);
-      if ((u & pmask) == prefix) atomicAdd(&sm.hist[(u >> shift) & 0xFFu], 1u);
-    }
+    src.visit([&](int, uint32_t u, int32_t t) {
+      if (!take(u, t)) return;
+      const uint32_t r = key(u, t) - kmin;
+      if ((r & pmask) == prefix) atomicAdd(&sm.hist[(r >> lo_bit) & dm], 1u);
+    });
     __syncthreads();
     if (tid < 32) {
       // lane l holds bins [8 (31 - l), 8 (31 - l) + 8): lane 0 the largest digits
@@ -122,17 +230,22 @@ __device__ uint32_t radix_kth(SelSmem& sm, int n, uint32_t k, Key key, Take take
       }
     }
     __syncthreads();
-    prefix |= sm.bin << shift;
-    pmask |= 0xFFu << shift;
+    prefix |= sm.bin << lo_bit;
+    pmask |= dm << lo_bit;
     remaining = sm.rem;
     eq = sm.eq;
     __syncthreads();   // sm.bin / sm.rem are rewritten by the next pass
+    if (lo_bit == 0) break;
+    top = lo_bit;
   }
   *need = remaining;
   *n_equal = eq;
-  return prefix;
+  return kmin + prefix;
 }
 
+// One CTA per query. P > 0: the row's candidates in registers (n <= P x 1024); P == 0:
+// MemCands.
+template <int P>
 __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSelectArgs a) {
   extern __shared__ uint8_t sel_smem_raw[];
   SelSmem& sm = *reinterpret_cast<SelSmem*>(sel_smem_raw);
@@ -144,17 +257,13 @@ __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSe
   pdl_trigger();
   pdl_wait();   // the gathered candidates may come from an earlier kernel on the stream
 
-  CandView v{a.all_score, a.all_token, nullptr, nullptr, K, a.Bq, q};
-  if (a.in_smem) {
-    uint32_t* skey = reinterpret_cast<uint32_t*>(sel_smem_raw + sizeof(SelSmem));
-    int32_t* stok = reinterpret_cast<int32_t*>(skey + n);
-    for (int c = tid; c < n; c += kSelThreads) {
-      const int64_t g = v.gidx(c);
-      skey[c] = order_key(a.all_score[g]);
-      stok[c] = a.all_token[g];
-    }
-    v.skey = skey;
-    v.stok = stok;
+  using Src = typename std::conditional<(P > 0), RegCands<(P > 0 ? P : 1)>, MemCands>::type;
+  Src src;
+  if constexpr (P > 0) {
+    src.load(a, n, q);
+  } else {
+    src = MemCands{a.all_score, a.all_token, nullptr, nullptr, n, K, a.Bq, q};
+    src.load(a, sel_smem_raw + sizeof(SelSmem));
   }
   if (tid == 0) {
     sm.n_valid = 0u;
@@ -165,7 +274,7 @@ __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSe
   __syncthreads();
   {
     uint32_t cnt = 0u;
-    for (int c = tid; c < n; c += kSelThreads) cnt += v.token(c) >= 0 ? 1u : 0u;
+    src.visit([&](int, uint32_t, int32_t t) { cnt += t >= 0 ? 1u : 0u; });
     cnt = __reduce_add_sync(0xffffffffu, cnt);
     if ((tid & 31) == 0 && cnt != 0u) atomicAdd(&sm.n_valid, cnt);
   }
@@ -175,18 +284,19 @@ __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSe
 
   // selection rule: all valid candidates (k == n_valid), else score key above kth, or equal
   // to it and among the `need` lowest global tokens of those equal
-  bool all = k == n_valid;
+  const bool all = k == n_valid;
   uint32_t kth = 0u, need = 0u, n_equal = 0u, kth2 = 0u, need2 = 0u, n_equal2 = 0u;
   bool all_equal = true;
-  auto valid = [&](int c) { return v.token(c) >= 0; };
   if (!all) {
-    kth = radix_kth(sm, n, k, [&](int c) { return v.key(c); }, valid, &need, &n_equal);
+    kth = radix_kth(
+        sm, src, k, [](uint32_t u, int32_t) { return u; }, [](uint32_t, int32_t t) { return t >= 0; }, &need,
+        &n_equal);
     all_equal = need == n_equal;
     if (!all_equal) {
       // ties at the k-th score: the `need` lowest tokens (larger key = lower token)
       kth2 = radix_kth(
-          sm, n, need, [&](int c) { return ~static_cast<uint32_t>(v.token(c)); },
-          [&](int c) { return valid(c) && v.key(c) == kth; }, &need2, &n_equal2);
+          sm, src, need, [](uint32_t, int32_t t) { return ~static_cast<uint32_t>(t); },
+          [kth](uint32_t u, int32_t t) { return t >= 0 && u == kth; }, &need2, &n_equal2);
     }
   }
 
@@ -195,11 +305,11 @@ __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSe
   len = len < 0 ? 0 : (len > a.max_pages * kPage ? a.max_pages * kPage : len);
   int32_t* lo_row = a.logical ? a.logical + static_cast<int64_t>(q) * K : nullptr;
   int32_t* ph_row = a.physical + static_cast<int64_t>(q) * K;
-  for (int c = tid; c < n; c += kSelThreads) {
-    const int tok = v.token(c);
+  // output positions come from one shared atomic per warp (ballot + popcount)
+  const unsigned lt_mask = (1u << (tid & 31)) - 1u;
+  src.visit([&](int c, uint32_t u, int32_t tok) {
     bool pick = tok >= 0;
     if (pick && !all) {
-      const uint32_t u = v.key(c);
       if (u < kth) {
         pick = false;
       } else if (u == kth && !all_equal) {
@@ -208,22 +318,43 @@ __global__ void __launch_bounds__(kSelThreads) shard_select_kernel(const ShardSe
         pick = u2 > kth2 || (u2 == kth2 && atomicAdd(&sm.n_eq2, 1u) < need2);
       }
     }
-    if (!pick) continue;
-    const uint32_t p = atomicAdd(&sm.n_sel, 1u);
-    if (p >= k) continue;
-    if (lo_row) lo_row[p] = tok;
-    if (c / K != a.rank) continue;
-    const int s = tok - off;
-    if (s < 0 || s >= len) {
-      record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(tok));
-      continue;
+    const unsigned picks = __ballot_sync(0xffffffffu, pick);
+    uint32_t base = 0u;
+    if ((tid & 31) == 0 && picks != 0u) base = atomicAdd(&sm.n_sel, static_cast<uint32_t>(__popc(picks)));
+    const uint32_t p = __shfl_sync(0xffffffffu, base, 0) + static_cast<uint32_t>(__popc(picks & lt_mask));
+    int local = -1;   // this rank's winners: local token now, its slot below
+    if (pick && p < k) {
+      if (lo_row) lo_row[p] = tok;
+      if (c / K == a.rank) {
+        const int s = tok - off;
+        if (s < 0 || s >= len) record_error(a.err, DSA_ERR_DEVICE_BOUNDS, static_cast<unsigned int>(tok));
+        else local = s;
+      }
     }
-    const int slot = checked_page(a.block_table, b, s >> 6, a.max_pages, a.num_pages, a.err) * kPage + (s & 63);
-    ph_row[atomicAdd(&sm.n_mine, 1u)] = slot;
-  }
+    const unsigned mine = __ballot_sync(0xffffffffu, local >= 0);
+    uint32_t mbase = 0u;
+    if ((tid & 31) == 0 && mine != 0u) mbase = atomicAdd(&sm.n_mine, static_cast<uint32_t>(__popc(mine)));
+    mbase = __shfl_sync(0xffffffffu, mbase, 0);
+    if (local >= 0) ph_row[mbase + __popc(mine & lt_mask)] = local;
+  });
   __syncthreads();
   const int n_sel = static_cast<int>(sm.n_sel < k ? sm.n_sel : k);
   const int n_mine = static_cast<int>(sm.n_mine);
+  // page map of this rank's winners, all block-table loads of a thread in flight together
+  constexpr int kU = 4;
+  for (int i0 = tid; i0 < n_mine; i0 += kU * kSelThreads) {
+    int s_[kU], pg[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) s_[u] = i0 + u * kSelThreads < n_mine ? ph_row[i0 + u * kSelThreads] : 0;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      pg[u] = i0 + u * kSelThreads < n_mine
+                  ? checked_page(a.block_table, b, s_[u] >> 6, a.max_pages, a.num_pages, a.err)
+                  : 0;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (i0 + u * kSelThreads < n_mine) ph_row[i0 + u * kSelThreads] = pg[u] * kPage + (s_[u] & 63);
+  }
   if (lo_row)
     for (int i = n_sel + tid; i < K; i += kSelThreads) lo_row[i] = -1;
   for (int i = n_mine + tid; i < K; i += kSelThreads) ph_row[i] = -1;
@@ -293,13 +424,19 @@ cudaError_t launch_shard_candidates(const ShardCandArgs& a, cudaStream_t stream,
 }
 
 cudaError_t launch_shard_select(const ShardSelectArgs& a, cudaStream_t stream, int* launches) {
-  const int smem = a.in_smem ? shard_select_smem_bytes(a.n_ranks * a.top_k) : static_cast<int>(sizeof(SelSmem));
+  const int n = a.n_ranks * a.top_k;
+  const dim3 grid(a.Bq), block(kSelThreads);
+  const int small = static_cast<int>(sizeof(SelSmem));
+  ++*launches;
+  if (n <= 4 * kSelThreads) return launch_pdl(shard_select_kernel<4>, grid, block, small, stream, a);
+  if (n <= 8 * kSelThreads) return launch_pdl(shard_select_kernel<8>, grid, block, small, stream, a);
+  if (n <= 16 * kSelThreads) return launch_pdl(shard_select_kernel<16>, grid, block, small, stream, a);
+  const int smem = a.in_smem ? shard_select_smem_bytes(n) : small;
   if (smem > 48 * 1024) {
-    const cudaError_t e = set_smem_once<shard_select_kernel>(kShardSelectSmemCap);
+    const cudaError_t e = set_smem_once<shard_select_kernel<0>>(kShardSelectSmemCap);
     if (e != cudaSuccess) return e;
   }
-  ++*launches;
-  return launch_pdl(shard_select_kernel, dim3(a.Bq), dim3(kSelThreads), smem, stream, a);
+  return launch_pdl(shard_select_kernel<0>, grid, block, smem, stream, a);
 }
 
 cudaError_t launch_shard_merge(const ShardMergeArgs& a, cudaStream_t stream, int* launches) {

@@ -23,7 +23,14 @@ CASES = {
     "bf16": CaseSpec("bf16", (1500, 129), top_k=128, idx_dtype="bf16", kv_dtype="bf16", out_dtype="fp32", seed=53),
     "packed_two_queries": CaseSpec("packed_two_queries", (2500, 900), top_k=256, kv_dtype="fp8r", n_q=2,
                                    n_planted=0, seed=54),
+    # 3 x 8192 candidates per query: the select's shared-memory copy; 4 x 8192: global reads
+    "wide_select": CaseSpec("wide_select", (40000,), top_k=8192, seed=55),
 }
+# (case, layout) pairs: every case on every layout except the wide one, which takes the two
+# layouts that reach the select's memory paths; 8 x 2048 candidates fill 16 registers a thread
+PAIRS = ([(n, l) for n in sorted(CASES) if n != "wide_select"
+          for l in ("even1", "even2", "even3", "even4", "uneven")]
+         + [("long_row", "even8"), ("wide_select", "even3"), ("wide_select", "even4")])
 
 
 @functools.lru_cache(maxsize=None)
@@ -110,8 +117,7 @@ def run_sharded(case, bounds):
     )
 
 
-@pytest.mark.parametrize("layout", ["even1", "even2", "even3", "even4", "uneven"])
-@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("name,layout", PAIRS)
 def test_sharded_decode(name, layout):
     case = get_case(name)
     bounds = _bounds(case, layout)
