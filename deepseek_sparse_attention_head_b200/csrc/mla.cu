@@ -863,22 +863,53 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
   const int g = t >> 5;                 // value group of dims 4 t .. 4 t + 3
   const int S = a.nsplit;
   const float* ml = a.part_ml + static_cast<int64_t>(q) * S * kHeads * kPartStats;
-  float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[(s * kHeads + h) * kPartStats]);
-  float Lsum = 0.0f, Lg = 0.0f;
+  // one pass over batches of eight splits, every load of a batch in flight together (a
+  // split at a time costs one L2 round trip each); the running max M rises batch by batch
+  // and what was summed so far is rescaled by 2^(M_old - M_new). A split that saw no valid
+  // row (m = -inf) contributes nothing, whatever its o holds.
+  constexpr int kB = 8;
+  float M = -INFINITY, Lsum = 0.0f, Lg = 0.0f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < S; ++s) {
-    const float* st = ml + (s * kHeads + h) * kPartStats;
-    const float m = st[0];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    Lsum += w * st[1];
-    Lg += w * st[2 + g];
-    const float4 o = reinterpret_cast<const float4*>(a.part_o + ((static_cast<int64_t>(q) * S + s) * kHeads + h) * kDimV)[t];
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
+  for (int s0 = 0; s0 < S; s0 += kB) {
+    float m[kB], l1[kB], lg[kB];
+    float4 o[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int s = s0 + u;
+      m[u] = -INFINITY;
+      l1[u] = lg[u] = 0.0f;
+      o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s < S) {
+        const float* st = ml + (s * kHeads + h) * kPartStats;
+        m[u] = st[0];
+        l1[u] = st[1];
+        lg[u] = st[2 + g];
+        o[u] = reinterpret_cast<const float4*>(a.part_o + ((static_cast<int64_t>(q) * S + s) * kHeads + h) * kDimV)[t];
+      }
+    }
+    float bm = M;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) bm = fmaxf(bm, m[u]);
+    if (bm == -INFINITY) continue;
+    const float c = exp2f(M - bm);   // 0 while nothing was summed (M = -inf)
+    Lsum *= c;
+    Lg *= c;
+    acc.x *= c;
+    acc.y *= c;
+    acc.z *= c;
+    acc.w *= c;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (m[u] == -INFINITY) continue;
+      const float w = exp2f(m[u] - bm);
+      Lsum += w * l1[u];
+      Lg += w * lg[u];
+      acc.x += w * o[u].x;
+      acc.y += w * o[u].y;
+      acc.z += w * o[u].z;
+      acc.w += w * o[u].w;
+    }
+    M = bm;
   }
   const float inv = Lg > 0.0f ? 1.0f / Lg : 0.0f;
   const float r[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
