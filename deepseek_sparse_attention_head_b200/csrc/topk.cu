@@ -158,8 +158,19 @@ __device__ uint32_t row_threshold(TopkSmem& sm, const float* row, int vis, int K
   constexpr int kMaxSamples = 4096;
   const int tid = threadIdx.x;
   const int S = min(kMaxSamples, vis);
-  for (int i = tid; i < S; i += kTopkThreads)
-    sm.cand_key[i] = order_key(__ldg(row + static_cast<int>((static_cast<int64_t>(i) * vis) / S)));
+  {
+    // all of a thread's samples in flight at once, then stored
+    constexpr int kPerT = kMaxSamples / kTopkThreads;
+    uint32_t sk[kPerT];
+#pragma unroll
+    for (int j = 0; j < kPerT; ++j) {
+      const int i = tid + j * kTopkThreads;
+      sk[j] = i < S ? order_key(__ldg(row + static_cast<int>((static_cast<int64_t>(i) * vis) / S))) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kPerT; ++j)
+      if (tid + j * kTopkThreads < S) sm.cand_key[tid + j * kTopkThreads] = sk[j];
+  }
   const float expect = static_cast<float>(S) * static_cast<float>(K) / static_cast<float>(vis);
   const uint32_t need = static_cast<uint32_t>(
       fminf(1.25f * expect + 3.0f * sqrtf(expect) + 4.0f, static_cast<float>(S)));
@@ -602,9 +613,27 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const TopkArg
   if (n_c >= static_cast<uint32_t>(rw.K) && n_c <= static_cast<uint32_t>(kCand) && n_c <= static_cast<uint32_t>(a.cand_cap)) {
     const uint32_t* gk = a.g_key + q * a.cand_cap;
     const int32_t* gi = a.g_idx + q * a.cand_cap;
-    for (int i = threadIdx.x; i < static_cast<int>(n_c); i += kTopkThreads) {
-      sm.cand_key[i] = gk[i];
-      sm.cand_idx[i] = gi[i];
+    // all of a thread's candidates in flight at once, then stored
+    constexpr int kPer = kCand / kTopkThreads;
+    uint32_t kk[kPer];
+    int32_t ii[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = static_cast<int>(threadIdx.x) + j * kTopkThreads;
+      kk[j] = 0u;
+      ii[j] = 0;
+      if (i < static_cast<int>(n_c)) {
+        kk[j] = __ldcg(gk + i);
+        ii[j] = __ldcg(gi + i);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = static_cast<int>(threadIdx.x) + j * kTopkThreads;
+      if (i < static_cast<int>(n_c)) {
+        sm.cand_key[i] = kk[j];
+        sm.cand_idx[i] = ii[j];
+      }
     }
     __syncthreads();
     select_and_emit(sm, a, rw, n_c, a.g_thr[q], a.g_rmax[q]);
