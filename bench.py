@@ -256,16 +256,25 @@ def time_stage(call, reps, nbytes, stream, flush):
             f"the call alone, L2 flushed before each ({nbytes / 1e6:.1f} MB < L2), mean of {reps}")
 
 
-def e2e_serial(t, in_keys, pin, host_out, host_lse, out, lse, step, stream, flush, n, use_graph, world):
+def e2e_serial(dsa, case, t, in_keys, pin, out, lse, ws, stream, flush, n, use_graph, world):
     """Device ms of n steps, each copy-in, layer call and copy-out in turn on one stream and
-    timed alone after an L2 flush (for workloads that fit in L2)."""
+    timed alone after an L2 flush (for workloads that fit in L2). Inputs and outputs cross
+    the host link as one packed copy each way (see Packed)."""
+    hin = Packed({k: t[k] for k in in_keys}, pinned=True)
+    for k in in_keys:
+        hin.views[k].copy_(pin[k])
+    hout = Packed({"out": out, "lse": lse}, pinned=True)
+    din = Packed({k: t[k] for k in in_keys}, device="cuda")
+    dout = Packed({"out": out, "lse": lse}, device="cuda")
+    dev = din.views
+    pg = dsa.Paging(dev["seq_lens"], dev["block_table"], case["num_pages"], case["n_q"], t["q_pos"])
 
     def body():
-        for k in in_keys:
-            t[k].copy_(pin[k], non_blocking=True)
-        step()
-        host_out.copy_(out, non_blocking=True)
-        host_lse.copy_(lse, non_blocking=True)
+        din.buf.copy_(hin.buf, non_blocking=True)
+        dsa.dsa_decode_layer(pg, dev["q_idx"], dev.get("q_idx_scale"), dev["head_w"], t["k_cache"], t["k_scale"],
+                             dev["q_mla"], t["kv_cache"], t["kv_scale"], case["top_k"], case["softmax_scale"],
+                             dout.views["out"], ws, lse=dout.views["lse"], stream=stream)
+        hout.buf.copy_(dout.buf, non_blocking=True)
 
     g = None
     if use_graph:
@@ -285,12 +294,29 @@ def e2e_serial(t, in_keys, pin, host_out, host_lse, out, lse, step, stream, flus
     ms = timed_flushed(call, n, stream, flush)
     torch.cuda.synchronize()
     del g
-    how = "serial steps from one CUDA graph each (copies included), L2 flushed before each" if use_graph else \
-        "serial eager steps (copies included), L2 flushed before each"
+    how = ("serial steps from one CUDA graph each (one packed copy each way included), L2 flushed before each"
+           if use_graph else "serial eager steps (one packed copy each way included), L2 flushed before each")
     return ms, how
 
 
-def e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, stream, n, use_graph, world):
+class Packed:
+    """Tensors laid out back to back (each at a 256-byte boundary) in one buffer, so that a
+    step's inputs, or its outputs, cross the host link as one copy: a few-MB copy reaches
+    the link's rate where several smaller ones each pay a fixed cost. `views[k]` is a
+    contiguous tensor of tensor k's dtype and shape inside the buffer."""
+
+    def __init__(self, like: dict, device=None, pinned=False):
+        spans, off = {}, 0
+        for k, v in like.items():
+            nb = v.numel() * v.element_size()
+            spans[k] = (off, nb)
+            off += (nb + 255) // 256 * 256
+        self.buf = torch.empty(off, dtype=torch.uint8, device=device, pin_memory=pinned)
+        self.views = {k: self.buf[o:o + nb].view(like[k].dtype).view(like[k].shape) for k, (o, nb) in spans.items()}
+        self.nbytes = off
+
+
+def e2e_pipelined(dsa, case, t, in_keys, pin, out, lse, ws, stream, n, use_graph, world):
     """Device ms from the first copy-in to the last copy-out of n steps over two buffer sets,
     as a serving loop overlaps them: while step k computes on set k % 2, step k+1's inputs
     are copied into the other set (its own stream) and step k-1's output and lse are copied
@@ -298,22 +324,30 @@ def e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, 
     joined) is one CUDA graph per set parity. The first stage's copy-out and the last
     stage's copy-in move bytes no step uses: n + 1 copies each way for n steps."""
     K = case["top_k"]
-    sets = []
+    # one pinned host buffer holds a step's inputs and one its outputs; every set of device
+    # buffers is packed the same way, so each direction is one copy per step
+    hin = Packed({k: t[k] for k in in_keys}, pinned=True)
+    for k in in_keys:
+        hin.views[k].copy_(pin[k])
+    hout = Packed({"out": out, "lse": lse}, pinned=True)
+    sets, packs = [], []
     for si in range(2):
-        dev = {k: (t[k] if si == 0 else t[k].clone()) for k in in_keys}
+        din = Packed({k: t[k] for k in in_keys}, device="cuda")
+        din.buf.copy_(hin.buf)
+        dout = Packed({"out": out, "lse": lse}, device="cuda")
+        dev = din.views
         pg = dsa.Paging(dev["seq_lens"], dev["block_table"], case["num_pages"], case["n_q"], t["q_pos"])
-        sets.append((dev, pg, out if si == 0 else torch.empty_like(out), lse if si == 0 else torch.empty_like(lse)))
+        sets.append((dev, pg, dout.views["out"], dout.views["lse"]))
+        packs.append((din, dout))
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
 
     def copy_in(si):
         with torch.cuda.stream(cin):
-            for k in in_keys:
-                sets[si][0][k].copy_(pin[k], non_blocking=True)
+            packs[si][0].buf.copy_(hin.buf, non_blocking=True)
 
     def copy_out(si):
         with torch.cuda.stream(cout):
-            host_out.copy_(sets[si][2], non_blocking=True)
-            host_lse.copy_(sets[si][3], non_blocking=True)
+            hout.buf.copy_(packs[si][1].buf, non_blocking=True)
 
     def stage(si):
         """Step on set si; the other set's inputs in and outputs out meanwhile."""
@@ -326,7 +360,7 @@ def e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, 
         copy_out(other)
         dev, pg, o, l = sets[si]
         with torch.cuda.stream(stream):
-            dsa.dsa_decode_layer(pg, dev["q_idx"], dev["q_idx_scale"], dev["head_w"], t["k_cache"], t["k_scale"],
+            dsa.dsa_decode_layer(pg, dev["q_idx"], dev.get("q_idx_scale"), dev["head_w"], t["k_cache"], t["k_scale"],
                                  dev["q_mla"], t["kv_cache"], t["kv_scale"], K, case["softmax_scale"], o, ws, lse=l,
                                  stream=stream)
         j_in, j_out = torch.cuda.Event(), torch.cuda.Event()
@@ -373,7 +407,8 @@ def e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, 
     ms = e0.elapsed_time(e1)
     del graphs
     how = ("pipelined over two buffer sets: copy-in of the next step and copy-out of the previous one overlap "
-           "each step, " + ("one CUDA graph per stage" if use_graph else "eager launches"))
+           "each step, one packed copy each way per step, " +
+           ("one CUDA graph per stage" if use_graph else "eager launches"))
     return ms, how
 
 
@@ -478,16 +513,14 @@ def run_ours(args, world, rank, local):
     # query-side inputs in from pinned host memory and its output and lse back out
     in_keys = [k for k in ("q_idx", "q_idx_scale", "head_w", "q_mla", "seq_lens", "block_table") if t[k] is not None]
     pin = {k: t[k].cpu().pin_memory() for k in in_keys}
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in pin.values())
-    d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
     n_e2e = max(10, args.e2e_steps)
     if inputs_exceed_l2:
-        e2e_local, e2e_how = e2e_pipelined(dsa, case, t, in_keys, pin, host_out, host_lse, out, lse, ws, stream,
-                                           n_e2e, graph is not None, world)
+        e2e_local, e2e_how = e2e_pipelined(dsa, case, t, in_keys, pin, out, lse, ws, stream, n_e2e,
+                                           graph is not None, world)
     else:
-        e2e_local, e2e_how = e2e_serial(t, in_keys, pin, host_out, host_lse, out, lse, step, stream, flush, n_e2e,
+        e2e_local, e2e_how = e2e_serial(dsa, case, t, in_keys, pin, out, lse, ws, stream, flush, n_e2e,
                                         graph is not None, world)
     e2e_ms = max_over_ranks(e2e_local, world)
 

@@ -73,3 +73,24 @@ def test_stage_timing_picks_by_bytes(clock):
     ms, how = bench.time_stage(_call(clock), 10, bench.L2_BYTES // 2, None, _Flush(clock))
     assert ms == pytest.approx(2.0) and "flushed" in how
     assert clock.log[:5] == ["call"] * 5 and clock.log[5:] == ["flush", "rec", "call", "rec"] * 10
+
+
+def test_packed_buffer_views_are_aligned_disjoint_and_typed():
+    import torch
+    like = {"a": torch.zeros(3, 5, dtype=torch.bfloat16), "b": torch.zeros(7, dtype=torch.int32),
+            "c": torch.zeros(2, 64, dtype=torch.uint8), "d": torch.zeros(1, dtype=torch.float32)}
+    p = bench.Packed(like)
+    spans = []
+    for k, v in like.items():
+        w = p.views[k]
+        assert w.dtype == v.dtype and w.shape == v.shape and w.is_contiguous()
+        off = w.data_ptr() - p.buf.data_ptr()
+        assert off % 256 == 0
+        spans.append((off, off + v.numel() * v.element_size()))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert p.nbytes == p.buf.numel() and spans[-1][1] <= p.nbytes
+    for i, (k, v) in enumerate(like.items()):
+        p.views[k].fill_(i + 1)
+    for i, k in enumerate(like):
+        assert torch.all(p.views[k] == i + 1)
