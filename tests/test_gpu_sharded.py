@@ -25,17 +25,29 @@ CASES = {
                                    n_planted=0, seed=54),
     # 3 x 8192 candidates per query: the select's shared-memory copy; 4 x 8192: global reads
     "wide_select": CaseSpec("wide_select", (40000,), top_k=8192, seed=55),
+    # a top_k that divides nothing, ragged rows
+    "odd_topk": CaseSpec("odd_topk", (1000, 333, 77), top_k=100, seed=56),
+    # every token's indexer key the same: all scores tie, so the global select takes its
+    # second radix pass (lowest global tokens among the candidates)
+    "all_ties": CaseSpec("all_ties", (3000, 500), top_k=256, seed=57),
 }
+TIED = {"all_ties"}
 # (case, layout) pairs: every case on every layout except the wide one, which takes the two
 # layouts that reach the select's memory paths; 8 x 2048 candidates fill 16 registers a thread
-PAIRS = ([(n, l) for n in sorted(CASES) if n != "wide_select"
+PAIRS = ([(n, l) for n in sorted(CASES) if n not in ("wide_select", "odd_topk", "all_ties")
           for l in ("even1", "even2", "even3", "even4", "uneven")]
-         + [("long_row", "even8"), ("wide_select", "even3"), ("wide_select", "even4")])
+         + [("long_row", "even8"), ("wide_select", "even3"), ("wide_select", "even4")]
+         + [(n, l) for n in ("odd_topk", "all_ties") for l in ("even1", "even3", "uneven")])
 
 
 @functools.lru_cache(maxsize=None)
 def get_case(name):
-    return generate(CASES[name])
+    case = generate(CASES[name])
+    if name in TIED:
+        case["k_cache"][:] = case["k_cache"][0, 0]
+        if case["k_scale"] is not None:
+            case["k_scale"][:] = case["k_scale"][0, 0]
+    return case
 
 
 @functools.lru_cache(maxsize=None)
