@@ -23,7 +23,7 @@
 namespace dsa {
 
 constexpr int kSelThreads = 1024;
-constexpr int kSelBins = 256;   // 8-bit radix digits, four passes per 32-bit key
+constexpr int kSelBins = 256;   // 8-bit radix digits: at most four passes per 32-bit key
 
 // ------------------------------------------------------------------ candidates
 

@@ -290,17 +290,53 @@ __device__ __forceinline__ uint32_t gather_takes(const float4 (&cur)[kGatherU / 
 // *rmax_addr to the largest key - thr. `cur` holds the first batch, loaded by
 // gather_load(row, lo_s, hi_s, cur) (so that its loads can be in flight while the caller
 // derives thr). Whole CTA; the trip count is CTA-uniform.
+// kBlock: `counter` and `rmax_addr` are in global memory and shared by many CTAs (the
+// long-row chunks), so the CTA reserves its slots with one atomic per batch (a warp-sum
+// scan in wsum[0..32]) and publishes its largest offset with one atomicMax; otherwise each
+// warp reserves its own (a shared or distributed-shared counter).
+template <bool kBlock = false>
 __device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr, uint32_t* counter,
                              uint32_t* out_key, int32_t* out_idx, uint32_t cap, uint32_t* rmax_addr,
-                             float4 (&cur)[kGatherU / 4]) {
+                             float4 (&cur)[kGatherU / 4], uint32_t* wsum = nullptr) {
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   uint32_t lmax = 0;
   float4 nxt[kGatherU / 4];
   for (int base = lo_s; base < hi_s; base += kGatherBatch) {
     if (base + kGatherBatch < hi_s) gather_load(row, base + kGatherBatch, hi_s, nxt);
     uint32_t takes = base + kGatherBatch <= hi_s ? gather_takes<true>(cur, base, hi_s, thr)
                                                   : gather_takes<false>(cur, base, hi_s, thr);
-    uint32_t c = warp_reserve(counter, static_cast<uint32_t>(__popc(takes)));
+    uint32_t c;
+    if constexpr (kBlock) {
+      const uint32_t n = static_cast<uint32_t>(__popc(takes));
+      uint32_t incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t w = wsum[lane];
+        uint32_t wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t t = __shfl_up_sync(0xffffffffu, wi, off);
+          if (lane >= off) wi += t;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, wi, 31);
+        uint32_t b0 = 0u;
+        if (lane == 0 && total != 0u) b0 = atomicAdd(counter, total);
+        b0 = __shfl_sync(0xffffffffu, b0, 0);
+        wsum[lane] = b0 + wi - w;   // this warp's first slot
+      }
+      __syncthreads();
+      c = wsum[warp] + incl - n;
+      __syncthreads();   // wsum is rewritten by the next batch
+    } else {
+      c = warp_reserve(counter, static_cast<uint32_t>(__popc(takes)));
+    }
     // only the taken keys (a few percent) are visited
     while (takes != 0u) {
       const int bit = __ffs(takes) - 1;
@@ -322,7 +358,16 @@ __device__ void gather_range(const float* row, int lo_s, int hi_s, uint32_t thr,
     for (int j = 0; j < kGatherU / 4; ++j) cur[j] = nxt[j];
   }
   const uint32_t wmax = __reduce_max_sync(0xffffffffu, lmax);
-  if ((tid & 31) == 0 && wmax != 0u) atomicMax(rmax_addr, wmax);
+  if constexpr (kBlock) {
+    if (lane == 0) wsum[warp] = wmax;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t bmax = __reduce_max_sync(0xffffffffu, wsum[lane]);
+      if (lane == 0 && bmax != 0u) atomicMax(rmax_addr, bmax);
+    }
+  } else {
+    if ((tid & 31) == 0 && wmax != 0u) atomicMax(rmax_addr, wmax);
+  }
 }
 
 // Exact selection among the n_c shared-memory candidates (all keys >= thr, n_c in
@@ -592,8 +637,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_gather_kernel(const TopkArg
   const uint32_t thr = row_threshold(sm, rw.row, rw.vis, rw.K);
   const int64_t q = rw.q;
   if (blockIdx.x == 0 && threadIdx.x == 0) a.g_thr[q] = thr;
-  gather_range(rw.row, lo_s, hi_s, thr, a.g_cnt + q, a.g_key + q * a.cand_cap, a.g_idx + q * a.cand_cap,
-               static_cast<uint32_t>(a.cand_cap), a.g_rmax + q, first);
+  gather_range<true>(rw.row, lo_s, hi_s, thr, a.g_cnt + q, a.g_key + q * a.cand_cap, a.g_idx + q * a.cand_cap,
+               static_cast<uint32_t>(a.cand_cap), a.g_rmax + q, first, sm.wsum);
 }
 
 // Long rows, part 2: one CTA per query selects exactly among the gathered candidates
