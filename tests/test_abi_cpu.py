@@ -209,3 +209,13 @@ def test_shard_bounds_are_page_aligned_and_cover_the_row():
             assert all(x % 64 == 0 or x == L for x in b)   # every shard starts on a page
     with pytest.raises(ValueError):
         shard_bounds(10, 0)
+
+
+def test_token_sharded_decode_rejects_causal_positions():
+    from types import SimpleNamespace
+    import torch
+    from deepseek_sparse_attention_head_b200.sharded import TokenShardedDecode
+    paging = SimpleNamespace(q_pos=torch.zeros(1, dtype=torch.int32), Bq=1, L_layer=64)
+    with pytest.raises(ValueError):
+        TokenShardedDecode(paging, torch.zeros(1, dtype=torch.int32), 8, 0.1, 0, 2)
+

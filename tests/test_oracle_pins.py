@@ -474,6 +474,16 @@ def test_sharded_step_equals_unsharded(layout):
         assert np.all(bounds[i][own[ok]] <= sel[ok]) and np.all(sel[ok] < bounds[i][own[ok] + 1])
 
 
+def test_sharded_step_equals_unsharded_with_two_queries_per_row():
+    case = generate(CaseSpec("t", (400, 150), top_k=48, n_q=2, n_planted=0, seed=33, kv_dtype="bf16"))
+    bounds = np.array([[0, 128, 256, 400], [0, 64, 64, 150]])
+    a = oracle.decode_layer(case)
+    b = oracle.sharded_decode_layer(case, bounds)
+    assert np.array_equal(a["logical"], b["logical"])
+    assert np.allclose(a["out"], b["out"], rtol=1e-12, atol=1e-14)
+    assert np.allclose(a["lse"], b["lse"], rtol=1e-12)
+
+
 def test_sharded_step_dense_rows_take_every_token():
     case = generate(CaseSpec("t", (100, 40), top_k=128, seed=32))
     r = oracle.sharded_decode_layer(case, np.array([[0, 64, 100], [0, 0, 40]]))
