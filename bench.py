@@ -2,11 +2,14 @@
 sparse decode) on one B200, or N independent replicas under torchrun.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg2] [--impl ours|reference]
+    python bench.py --workload cfg3 --token-shards R [--gpus R]
 
 Prints one JSON line (rank 0). A step is one dsa_decode_layer call over the whole
 batch of the workload, with inputs resident in HBM. Workloads larger than L2 are timed
 as back-to-back steps; smaller ones, and the stages timed alone, get an L2 flush before
-every call, outside the timed intervals.
+every call, outside the timed intervals. --token-shards R times the token-sharded step
+instead: every row's tokens over R ranks, with two all-gathers (strong scaling); on one
+GPU the R ranks run in lockstep in one process.
 """
 from __future__ import annotations
 
@@ -52,9 +55,10 @@ def parse():
 # ------------------------------------------------------------------ distributed plumbing
 
 def dist_setup(args, backend=None):
-    """One process per GPU (torchrun env). The path shards by rows with no data-path
-    collective: every rank runs its own replica of the workload, and the process group
-    only carries the barriers and the max-over-ranks timing. NCCL on GPUs; gloo when
+    """One process per GPU (torchrun env). By default the path shards by rows with no
+    data-path collective: every rank runs its own replica of the workload, and the process
+    group only carries the barriers and the max-over-ranks timing. With --token-shards the
+    group also carries the token-sharded step's two all-gathers. NCCL on GPUs; gloo when
     asked for (the CPU tests) or when no GPU is present."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
