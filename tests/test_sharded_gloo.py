@@ -1,4 +1,4 @@
-"""The token-sharded step's host logic on CPU: two gloo ranks run TokenShardedDecode.step
+"""The token-sharded step's host logic on CPU: two or three gloo ranks run TokenShardedDecode.step
 with its real exchanges (all-gathers over the process group) while the library calls it
 makes are replaced, in the child processes of this test only, by fp64 oracle stand-ins of
 each stage. The merged output must be the oracle's sharded (and unsharded) step on every
@@ -10,6 +10,7 @@ import sys
 from types import SimpleNamespace
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -104,11 +105,15 @@ def _rank(rank, world, port, bounds, out):
     dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_merge_to_the_unsharded_step():
+@pytest.mark.parametrize("bounds", [
+    [[0, 192, 300], [0, 0, 130]],                  # two ranks; row 1 lives on rank 1 only
+    [[0, 64, 256, 300], [0, 128, 128, 130]],       # three ranks; rank 1 holds none of row 1
+], ids=["two_ranks", "three_ranks"])
+def test_gloo_ranks_merge_to_the_unsharded_step(bounds):
     import oracle
     from dsa_inputs import CaseSpec, generate
-    bounds = np.array([[0, 192, 300], [0, 0, 130]], dtype=np.int64)   # row 1 lives on rank 1 only
-    world = 2
+    bounds = np.array(bounds, dtype=np.int64)
+    world = bounds.shape[1] - 1
     with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank, args=(world, _free_port(), bounds, out), nprocs=world, join=True)
@@ -122,4 +127,5 @@ def test_two_gloo_ranks_merge_to_the_unsharded_step():
         assert np.array_equal(logical.astype(np.int64), ref["logical"])
         assert np.allclose(o, ref["out"], rtol=1e-5, atol=1e-6)
         assert np.allclose(lse, ref["lse"], rtol=1e-6)
-    assert np.array_equal(res[0][0], res[1][0])
+    for r in range(1, world):
+        assert np.array_equal(res[r][0], res[0][0])
