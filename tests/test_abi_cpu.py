@@ -113,6 +113,10 @@ def test_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError):
         dsa._ptr(torch.zeros(4))
+    # the token-sharded entry points marshal through the same checks: no host tensor reaches
+    # the library, and nothing falls back to a CPU computation
+    with pytest.raises(ValueError):
+        dsa.dsa_shard_merge(torch.zeros(2, 1, 64, 512), torch.zeros(2, 1, 64), torch.zeros(1, 64, 512))
 
 
 def test_noalloc_argument_errors():
